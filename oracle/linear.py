@@ -1,0 +1,68 @@
+"""fp64 definitions of the QLoRA linear layer forward and backward.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+Row-vector convention: W is [N, K] (out x in), X [M, K], A [K, r], B [r, N],
+s = alpha / r.  "QLoRA" (ozercemkelahmet.com), How it works, Step 5 writes the
+column form y = dequant(W) x + (alpha/r) B (A x); for token rows x^T this is
+Y = X deq(W)^T + s (X A') B' with A' = A, B' = B in [K, r] / [r, N] layout.
+Step 6: gradients flow through the dequantized weights into the adapters only;
+no gradient for W.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .nf4 import bf16_to_f32
+
+
+def as_f64(bits_or_f) -> np.ndarray:
+    a = np.asarray(bits_or_f)
+    if a.dtype == np.uint16:
+        return bf16_to_f32(a).astype(np.float64).reshape(a.shape)
+    return a.astype(np.float64)
+
+
+def forward(X, Wd, A, B, s: float):
+    """XA = X A;  Y = X Wd^T + s XA B.  All fp64; inputs may be bf16 bits."""
+    X, Wd, A, B = (as_f64(t) for t in (X, Wd, A, B))
+    XA = X @ A
+    Y = X @ Wd.T + s * (XA @ B)
+    return Y, XA
+
+
+def backward(dY, X, Wd, A, B, s: float, XA=None):
+    """G = dY B^T;  dX = dY Wd + s G A^T;  dA = s X^T G;  dB = s XA^T dY."""
+    dY, X, Wd, A, B = (as_f64(t) for t in (dY, X, Wd, A, B))
+    if XA is None:
+        XA = X @ A
+    else:
+        XA = np.asarray(XA, np.float64)
+    G = dY @ B.T
+    dX = dY @ Wd + s * (G @ A.T)
+    dA = s * (X.T @ G)
+    dB = s * (XA.T @ dY)
+    return dict(G=G, dX=dX, dA=dA, dB=dB)
+
+
+def forward_rows(X, Wd, A, B, s: float, rows):
+    """Y restricted to the given token rows (for sampled checks at full size)."""
+    rows = np.asarray(rows)
+    Y, XA = forward(as_f64(X)[rows], Wd, A, B, s)
+    return Y, XA
+
+
+def backward_rows_dx(dY, Wd, A, B, s: float, rows):
+    """dX restricted to the given token rows."""
+    dY = as_f64(dY)[np.asarray(rows)]
+    Wd, A, B = (as_f64(t) for t in (Wd, A, B))
+    G = dY @ B.T
+    return dY @ Wd + s * (G @ A.T)
+
+
+def rel_fro(got, ref) -> float:
+    """||got - ref||_F / ||ref||_F."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
