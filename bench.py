@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 frozen-base linear layer on B200.
+
+One step = forward + backward of the three LLaMA-7B-shaped adapted projections
+(W 4096x4096, 11008x4096, 4096x11008 stored as NF4 with double-quantized
+constants; 4096 tokens per GPU; LoRA r=16, alpha=32): per projection
+Y = X deq(W)^T + s (X A) B, then dX, dA, dB.  Weights are quantized once before
+timing (model load).  Metric: fwd+bwd TFLOP/s of algorithmic FLOPs
+4MNK + 6Mr(K+N) per projection.  Multi-GPU: data-parallel replicas (weak
+scaling), each rank its own 4096 tokens, dA/dB all-reduced over NCCL each step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4-weight HBM GB/s vs roofline, 1 B200"
+SHAPES = [(4096, 4096, 4096), (4096, 11008, 4096), (4096, 4096, 11008)]   # (M, N, K)
+RANK_R, ALPHA, W_STD = 16, 32.0, 0.02
+WORKLOAD = ("LLaMA-7B-shaped projections W[N,K] in {4096x4096, 11008x4096, 4096x11008}, NF4 "
+            "block 64 / double-quant 256; 4096 tokens per GPU; LoRA r=16 alpha=32; fwd+bwd")
+FLUSH_BYTES = 256 << 20
+SKINNY = [(m, n, 4096) for n in (4096, 11008) for m in (1, 4, 16)]
+BIG_N = 1_000_000_000
+
+
+def step_flops(M, N, K, r):
+    return 4.0 * M * N * K + 6.0 * M * r * (K + N)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_19_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key):
+    """dram bytes per launch from a committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t.get(kernel_key)
+        if e and e.get("source_hash") == source_hash():
+            return e.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/qlora_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        try:
+            rows = [l.strip().split(", ") for l in open(self.path) if l.strip()]
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_sample(problems, tokens, wrows, repeats=1):
+    """Oracle fwd+bwd on a bounded sample of every projection: the first
+    `tokens` tokens and the first `wrows` output features (dequant of those W
+    rows included, as the method dequantizes every step).  Returns (flops, s)."""
+    from oracle import linear as olin, nf4 as onf4
+    quant = []
+    for p in problems:
+        rows_q = onf4.quantize_bf16(p["W"][:wrows].ravel())
+        quant.append(rows_q)
+    flops, t0 = 0.0, time.perf_counter()
+    for _ in range(repeats):
+        for p, q in zip(problems, quant):
+            N, K = wrows, p["K"]
+            Wd = onf4.dequantize(q["codes"], q["q8"], q["step"], N * K).reshape(N, K)
+            X, A, B, dY = p["X"][:tokens], p["A"], p["B"][:, :wrows], p["dY"][:tokens, :wrows]
+            Y, XA = olin.forward(X, Wd, A, B, p["s"])
+            olin.backward(dY, X, Wd, A, B, p["s"], XA=XA)
+            flops += step_flops(tokens, N, K, p["r"])
+    return flops, time.perf_counter() - t0
+
+
+def cpu_info():
+    cores = len(os.sched_getaffinity(0))
+    blas = None
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 0) for i in threadpool_info()), default=None)
+    except Exception:
+        pass
+    return cores, blas
+
+
+def host_problems(seed):
+    from synth import linear_problem
+    out = []
+    for (M, N, K) in SHAPES:
+        p = linear_problem(M, N, K, RANK_R, ALPHA, W_STD, seed=0)      # frozen W: same on all ranks
+        if seed:
+            q = linear_problem(M, N, K, RANK_R, ALPHA, W_STD, seed=seed)
+            p.X, p.dY = q.X, q.dY                                      # per-rank tokens
+        out.append(dict(M=M, N=N, K=K, r=RANK_R, s=ALPHA / RANK_R, W=p.W, X=p.X, A=p.A, B=p.B,
+                        dY=p.dY))
+    return out
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    problems = host_problems(0)
+    tokens, wrows = 128, 512
+    for _ in range(max(0, args.warmup)):
+        oracle_sample(problems, tokens, wrows)
+    fl, t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, s = oracle_sample(problems, tokens, wrows)
+        fl += f
+        t += s
+    cores, blas = cpu_info()
+    v = fl / t / 1e12
+    sample = (f"oracle (NumPy/SciPy, fp64 GEMMs) per step: all 3 projections, first {tokens} "
+              f"tokens x first {wrows} output features, dequant of those rows included")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas or cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-subpaths", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import bit_nf4_quantized_19_b200 as q
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    hp = host_problems(rank)
+    P = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- device-resident state (weights quantized once, like a model load)
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    layers = []
+    grad_numel = sum(K * RANK_R + RANK_R * N for (_, N, K) in SHAPES)
+    flat_grads = torch.zeros(grad_numel, dtype=torch.float32, device=dev)
+    flat_host = torch.empty(grad_numel, dtype=torch.float32).pin_memory()
+    off = 0
+    for p in hp:
+        M, N, K, r = p["M"], p["N"], p["K"], p["r"]
+        Wq = q.nf4_quantize(to_dev(p["W"]))
+        L = dict(M=M, N=N, K=K, r=r, s=p["s"], Wq=Wq, X=to_dev(p["X"]), dY=to_dev(p["dY"]),
+                 A=to_dev(p["A"]), B=to_dev(p["B"]),
+                 Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                 XA=torch.empty(M, r, dtype=torch.float32, device=dev),
+                 dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+                 dA=flat_grads[off:off + K * r].view(K, r),
+                 dB=flat_grads[off + K * r:off + K * r + r * N].view(r, N),
+                 ws=q.make_workspace(M, N, K, r, dev))
+        off += K * r + r * N
+        L["hX"] = torch.from_numpy(np.ascontiguousarray(p["X"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        L["hdY"] = torch.from_numpy(np.ascontiguousarray(p["dY"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        layers.append(L)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        for L in layers:
+            q.linear_fwd(L["X"], L["Wq"], L["A"], L["B"], L["s"], workspace=L["ws"], Y=L["Y"],
+                         XA=L["XA"])
+            q.linear_bwd(L["dY"], L["X"], L["XA"], L["Wq"], L["A"], L["B"], L["s"],
+                         workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
+        if world > 1:
+            dist.all_reduce(flat_grads)
+
+    flops_per_step_rank = sum(step_flops(M, N, K, RANK_R) for (M, N, K) in SHAPES)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, flags = q.device_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} flags {flags} after warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each, CUDA events per step
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    q.profile_enable(True)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+    prof, nlaunch = q.profile_read()
+    q.profile_enable(False)
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    code, flags = q.device_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} flags {flags} after timing")
+    value = world * flops_per_step_rank * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- per-kernel breakdown and the dominant kernel's roofline
+    by = {}
+    for kind, ms in prof:
+        d = by.setdefault(kind, [0, 0.0])
+        d[0] += 1
+        d[1] += ms
+    kern_total = sum(v[1] for v in by.values()) or 1.0
+    kernels = {k: {"launches": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / kern_total, 4)}
+               for k, v in sorted(by.items(), key=lambda kv: -kv[1][1])}
+    gemm_flops = args.steps * sum(2.0 * M * N * K + 2.0 * M * N * RANK_R + 2.0 * M * N * K
+                                  + 2.0 * M * K * RANK_R for (M, N, K) in SHAPES)
+    gemm_ms = by.get("gemm_fwd", [0, 0.0])[1] + by.get("gemm_dx", [0, 0.0])[1]
+    gemm_launches = by.get("gemm_fwd", [0, 0.0])[0] + by.get("gemm_dx", [0, 0.0])[0]
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    roof = {"kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05 GEMM + LoRA K-steps; fwd and dX)",
+            "bound": "tensor", "achieved": achieved, "peak": P["bf16_sus"], "unit": "TFLOP/s",
+            "frac": (achieved / P["bf16_sus"]) if achieved else None,
+            "peak_source": f"{P['src']} bf16 sustained (MEASURED_PEAKS.json)",
+            "avg_launch_ms": gemm_ms / max(1, gemm_launches),
+            "traffic": traffic_for("qlora_gemm_kernel")}
+
+    # ---- end to end through the public API: pinned host inputs -> device -> grads back
+    e2e_steps = max(3, min(args.steps, 30))
+    h2d = sum(L["hX"].numel() * 2 + L["hdY"].numel() * 2 for L in layers)
+    d2h = flat_host.numel() * 4
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        for L in layers:
+            L["X"].copy_(L["hX"], non_blocking=True)
+            L["dY"].copy_(L["hdY"], non_blocking=True)
+        step()
+        flat_host.copy_(flat_grads, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * flops_per_step_rank * e2e_steps / (e2e_ms * 1e-3) / 1e12,
+           "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "steps": e2e_steps}
+
+    # ---- HBM-bound subpaths (quantize / dequant of 1e9 values, skinny forward)
+    subpaths = None
+    if not args.no_subpaths:
+        subpaths = hbm_subpaths(q, torch, dev, stream, P, flush)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        hp0 = host_problems(0)
+        tokens, wrows = 512, 2048
+        fl, sec = oracle_sample(hp0, tokens, wrows)
+        cores, blas = cpu_info()
+        cpu_baseline = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": blas or cores,
+                        "kind": "oracle",
+                        "sample": f"all 3 projections, first {tokens} tokens x first {wrows} "
+                                  f"output features, dequant of those rows included; {sec:.1f} s"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded): W ~ N(0,0.02) bf16 quantized to NF4, X, dY ~ N(0,1), "
+                        "A ~ N(0,1/r), B ~ N(0,0.01)",
+                "config": {"workload": WORKLOAD, "global_batch": 4096 * world,
+                           "tokens_per_gpu": 4096, "parallelism": f"dp{world}",
+                           "l2": "flushed (256 MiB write) before every timed step",
+                           "flops_per_step_per_gpu": flops_per_step_rank},
+                "roofline": roof, "cpu_baseline": cpu_baseline, "e2e": e2e,
+                "gpu_launches": nlaunch, "clocks": clk.summary(), "kernels": kernels,
+                "subpaths": subpaths}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def hbm_subpaths(q, torch, dev, stream, P, flush):
+    out = {}
+    # 1e9-value heavy-tailed tensor, generated on the device (seeded)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    W = torch.empty(BIG_N, dtype=torch.bfloat16, device=dev)
+    chunk = 1 << 26
+    for i in range(0, BIG_N, chunk):
+        n = min(chunk, BIG_N - i)
+        z = torch.randn(n, generator=g, device=dev, dtype=torch.float32) * 0.02
+        m = torch.rand(n, generator=g, device=dev) < 1e-3
+        z[m] *= 8.0
+        W[i:i + n] = z.to(torch.bfloat16)
+    del z, m
+    Wq = q.nf4_quantize(W.view(1, BIG_N))
+    out_bf = torch.empty(BIG_N, dtype=torch.bfloat16, device=dev)
+    q.nf4_dequant(Wq, out_bf.view(1, BIG_N))
+    torch.cuda.synchronize()
+    nbytes = BIG_N * 2 + Wq.nbytes
+    q.profile_enable(True)
+    for _ in range(3):
+        q.nf4_quantize(W.view(1, BIG_N), out=Wq)
+        q.nf4_dequant(Wq, out_bf.view(1, BIG_N))
+    prof, _ = q.profile_read()
+    q.profile_enable(False)
+    tq = min(ms for k, ms in prof if k == "quantize")
+    td = min(ms for k, ms in prof if k == "dequant")
+    out["quantize_1e9"] = {"ms": tq, "GB/s": nbytes / tq / 1e6, "frac": nbytes / tq / 1e6 / P["hbm"],
+                           "bytes": nbytes}
+    out["dequant_1e9"] = {"ms": td, "GB/s": nbytes / td / 1e6, "frac": nbytes / td / 1e6 / P["hbm"],
+                          "bytes": nbytes}
+    del W, Wq, out_bf
+    torch.cuda.empty_cache()
+    # skinny forward: M in {1,4,16}, L2 flushed before each call, whole call timed
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    for (M, N, K) in SKINNY:
+        r = RANK_R
+        Wb = (torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        Wq = q.nf4_quantize(Wb)
+        X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
+        A = (torch.randn(K, r, generator=gen, device=dev) / r).to(torch.bfloat16)
+        B = (torch.randn(r, N, generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        XA = torch.empty(M, r, dtype=torch.float32, device=dev)
+        ws = q.make_workspace(M, N, K, r, dev)
+        for _ in range(3):
+            q.linear_fwd(X, Wq, A, B, r and 2.0, workspace=ws, Y=Y, XA=XA)
+        ts = []
+        for i in range(20):
+            flush.fill_(float(i))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            q.linear_fwd(X, Wq, A, B, 2.0, workspace=ws, Y=Y, XA=XA)
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        t = statistics.median(a.elapsed_time(b) for a, b in ts)
+        by = Wq.nbytes + 2 * M * K + 2 * M * N + 2 * K * r + 2 * r * N + 4 * M * r
+        out[f"skinny_M{M}_{N}x{K}"] = {"ms": t, "GB/s": by / t / 1e6, "frac": by / t / 1e6 / P["hbm"],
+                                       "bytes": by}
+        del Wb, Wq
+    out["hbm_peak_GBps"] = P["hbm"]
+    out["hbm_peak_source"] = P["src"]
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,349 @@
+// Dequant-fused tcgen05 GEMM for the QLoRA linear layer (sm_100a).
+//
+// Forward ("QLoRA", ozercemkelahmet.com, How it works, Step 5; essay at
+// fanfani.net, "store in four bits, compute in sixteen"):
+//     Y^T[n, m] = sum_k deq(W)[n, k] X[m, k]  +  sum_c B'[n, c] XAhl[m, c]
+// dX (Step 6: gradients flow through the dequantized weights):
+//     dX^T[k, m] = sum_n deq(W)[n, k] dY[m, n] +  sum_c A'[k, c] Ghl[m, c]
+//
+// The weight side is the MMA's A operand (M = 128 weight rows or columns per
+// tile) and the tokens are the MMA's N (BN = 256 per tile), so every
+// dequantized value feeds 256 tokens.  The rank-r LoRA term is appended as
+// extra K steps in the same TMEM accumulator: the activation side carries
+// s*XA (or s*G) split into bf16 hi and lo halves (c < r: hi, r <= c < 2r: lo)
+// and the weight side repeats B^T (or A) twice, so the adapter term is
+// accumulated to ~2^-16 relative precision, not bf16 precision.
+//
+// Warp roles (384 threads, one CTA per SM, persistent over tiles):
+//   warp 0        TMA producer: activation tiles (X / dY, or the LoRA hi/lo
+//                 operand) and packed 4-bit weight tiles + block constants.
+//   warp 1        TMEM allocator and single-thread MMA issuer.
+//   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
+//   warps 8..11   dequant producers: packed codes + constant -> bf16 tile in
+//                 the 128-byte-swizzled UMMA layout, then LoRA weight tiles.
+// Every wait is bounded (see Waiter); a wait that runs out aborts the block.
+#pragma once
+#include "common.cuh"
+
+namespace qlora {
+
+constexpr int kGemmThreads = 384;
+constexpr int kBN = 256;                  // tokens per tile (MMA N)
+constexpr int kWT = 128;                  // weight-side rows per tile (MMA M)
+constexpr int kBK = 64;                   // contraction per stage (one quant block)
+constexpr int kStagesB = 4;               // activation ring
+constexpr int kStagesA = 3;               // dequantized weight ring
+constexpr int kStagesW = 4;               // packed code ring
+constexpr int kBStageBytes = kBN * 128;   // 32 KB
+constexpr int kAStageBytes = kWT * 128;   // 16 KB
+constexpr int kWStageBytes = 4096;        // packed codes of one stage
+constexpr int kSStageBytes = 512;         // 128 fp32 block constants of one stage
+constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
+
+constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStagesB * kBStageBytes +
+                               kStagesA * kAStageBytes + kStagesW * (kWStageBytes + kSStageBytes) +
+                               1024 /*barriers, flags, levels*/;
+
+enum GemmMode : int { kModeFwd = 0, kModeDx = 1 };
+
+struct GemmParams {
+  int M;             // tokens
+  int n_out;         // output row length (N for fwd, K for dX)
+  int num_m_tiles;   // ceil(M / 256)
+  int num_w_tiles;   // weight-side tiles: N/128 (fwd) or K/128 (dX)
+  int kb_main;       // main stages: K/64 (fwd) or N/64 (dX)
+  int kb_lora;       // LoRA stages: ceil(2r / 64)
+  int r;
+  int lora_ld;       // row pitch of the LoRA weight operand source: N (B [r,N]) or r (A [K,r])
+  const uint16_t *lora_w;  // fwd: B [r, N];  dX: A [K, r]
+  uint16_t *out;     // Y [M, N] or dX [M, K]
+  uint64_t limit_ns;
+  float levels[16];
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,   // X or dY, bf16 [M, contraction]
+                      const __grid_constant__ CUtensorMap tm_codes, // packed codes, u8 [N, K/2]
+                      const __grid_constant__ CUtensorMap tm_scale, // block constants, f32 [K/64, N]
+                      const __grid_constant__ CUtensorMap tm_lora,  // hi/lo LoRA operand, bf16 [M, 2r]
+                      const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sB = smem;
+  uint8_t *sA = sB + kStagesB * kBStageBytes;
+  uint8_t *sW = sA + kStagesA * kAStageBytes;
+  float *sS = reinterpret_cast<float *>(sW + kStagesW * kWStageBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sS + kStagesW * (kSStageBytes / 4));
+  uint64_t *full_B = bars;
+  uint64_t *empty_B = full_B + kStagesB;
+  uint64_t *full_A = empty_B + kStagesB;
+  uint64_t *empty_A = full_A + kStagesA;
+  uint64_t *full_W = empty_A + kStagesA;
+  uint64_t *empty_W = full_W + kStagesW;
+  uint64_t *tmem_full = empty_W + kStagesW;
+  uint64_t *tmem_empty = tmem_full + 2;
+  uint64_t *drain = tmem_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  float *sL = reinterpret_cast<float *>(abort_flag + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStagesB; ++i) { mbar_init(&full_B[i], 1); mbar_init(&empty_B[i], 1); }
+    for (int i = 0; i < kStagesA; ++i) { mbar_init(&full_A[i], 128); mbar_init(&empty_A[i], 1); }
+    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 1); mbar_init(&empty_W[i], 128); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 128); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < 16) sL[tid] = p.levels[tid];
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_act);
+    prefetch_tmap(&tm_codes);
+    prefetch_tmap(&tm_scale);
+    prefetch_tmap(&tm_lora);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const Waiter wt{abort_flag, p.limit_ns};
+
+  const int num_tiles = p.num_m_tiles * p.num_w_tiles;
+  const int nkb = p.kb_main + p.kb_lora;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int bs = 0, ws = 0;
+      uint32_t bph = 0, wph = 0;
+      uint32_t armedB = 0, armedW = 0;          // bit s: stage s armed at least once
+      uint32_t lastB = 0, lastW = 0;            // bit s: parity of the last arming
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int m0 = (tile / p.num_w_tiles) * kBN;
+        const int w0 = (tile % p.num_w_tiles) * kWT;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bar(&empty_B[bs], bph ^ 1u, wt)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_B[bs], kBStageBytes);
+          if (kb < p.kb_main)
+            tma_load_2d(sB + bs * kBStageBytes, &tm_act, &full_B[bs], kb * kBK, m0);
+          else
+            tma_load_2d(sB + bs * kBStageBytes, &tm_lora, &full_B[bs], (kb - p.kb_main) * kBK, m0);
+          armedB |= 1u << bs;
+          lastB = (lastB & ~(1u << bs)) | (bph << bs);
+          if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
+          if (kb < p.kb_main) {
+            if (!wait_bar(&empty_W[ws], wph ^ 1u, wt)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full_W[ws], kWStageBytes + kSStageBytes);
+            if (MODE == kModeFwd) {
+              // codes: 32 bytes (64 values of K) x 128 weight rows; constants S[kb][w0 .. w0+128)
+              tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
+              tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], w0, kb);
+            } else {
+              // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..;
+              // constants S[w0/64 + {0,1}][kb*64 .. kb*64+64)
+              tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
+              tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], kb * kBK, w0 / kBK);
+            }
+            armedW |= 1u << ws;
+            lastW = (lastW & ~(1u << ws)) | (wph << ws);
+            if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
+          }
+        }
+      }
+      // Every issued copy lands before the block may exit (bounded).
+      volatile int no_abort = 0;
+      const Waiter final_wt{&no_abort, p.limit_ns};
+      for (int s = 0; s < kStagesB; ++s)
+        if (armedB & (1u << s)) wait_bar(&full_B[s], (lastB >> s) & 1u, final_wt);
+      for (int s = 0; s < kStagesW; ++s)
+        if (armedW & (1u << s)) wait_bar(&full_W[s], (lastW >> s) & 1u, final_wt);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main = make_idesc_bf16(kWT, kBN, MODE == kModeDx, false);
+      constexpr uint32_t idesc_lora = make_idesc_bf16(kWT, kBN, MODE == kModeFwd, false);
+      int as = 0, bs = 0, acc = 0;
+      uint32_t aph = 0, bph = 0, accph = 0;
+      bool ok = true;
+      const int lora_steps_total = (2 * p.r) / 16;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!wait_bar(&tmem_empty[acc], accph ^ 1u, wt)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bar(&full_A[as], aph, wt) || !wait_bar(&full_B[bs], bph, wt)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + as * kAStageBytes);
+          const uint32_t b_base = smem_u32(sB + bs * kBStageBytes);
+          const bool main = kb < p.kb_main;
+          int nk = 4;
+          if (!main) {
+            const int done = (kb - p.kb_main) * 4;
+            nk = min(4, lora_steps_total - done);
+          }
+          for (int k = 0; k < nk; ++k) {
+            const bool a_mn = main ? (MODE == kModeDx) : (MODE == kModeFwd);
+            const uint64_t adesc = a_mn ? sw128_desc(a_base + k * 4096, 1024, 2048)
+                                        : sw128_desc(a_base + k * 32, 16, 1024);
+            const uint64_t bdesc = sw128_desc(b_base + k * 32, 16, 1024);
+            mma_bf16_ss(d_tmem, adesc, bdesc, main ? idesc_main : idesc_lora,
+                        (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty_A[as]);
+          mma_commit(&empty_B[bs]);
+          if (++as == kStagesA) { as = 0; aph ^= 1u; }
+          if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tmem_full[acc]);
+        if (++acc == 2) { acc = 0; accph ^= 1u; }
+      }
+      // All issued MMAs complete before TMEM is released (bounded).
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      const Waiter final_wt{&no_abort, p.limit_ns};
+      wait_bar(drain, 0, final_wt);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;             // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;      // weight-side row within the tile
+    int acc = 0;
+    uint32_t accph = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m0 = (tile / p.num_w_tiles) * kBN;
+      const int w0 = (tile % p.num_w_tiles) * kWT;
+      // warp-uniform decision: the TMEM loads below are .sync.aligned
+      const bool got = __all_sync(0xffffffffu, wait_bar(&tmem_full[acc], accph, wt) ? 1 : 0);
+      if (!got) break;
+      tc_fence_after();
+      uint16_t *outc = p.out + w0 + row;
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * kBN + cc * 32),
+                           v);
+        tmem_wait_ld();
+        const int mb = m0 + cc * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int m = mb + j;
+          if (m < p.M) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[j]));
+            outc[static_cast<int64_t>(m) * p.n_out] = *reinterpret_cast<const uint16_t *>(&h);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tmem_empty[acc]);
+      if (++acc == 2) { acc = 0; accph ^= 1u; }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dequant producers
+    const int t = tid - 256;            // 0..127
+    int as = 0, ws = 0;
+    uint32_t aph = 0, wph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const int w0 = (tile % p.num_w_tiles) * kWT;
+      for (int kb = 0; kb < p.kb_main; ++kb) {
+        if (!wait_bar(&full_W[ws], wph, wt) || !wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+        // Which block this thread expands and where its 128-byte row goes.
+        uint32_t src, dst;
+        int swz;
+        float sc;
+        if (MODE == kModeFwd) {
+          // row t of the tile: weight row w0+t, 64 values of K (one block)
+          src = smem_u32(sW + ws * kWStageBytes + t * 32);
+          sc = sS[ws * 128 + t];
+          dst = smem_u32(sA + as * kAStageBytes + t * 128);
+          swz = t & 7;
+        } else {
+          // weight row n = kb*64 + nl, 64 values of K starting at w0 + 64*kk;
+          // MN-major: K index nl, M group kk
+          const int nl = t & 63, kk = t >> 6;
+          src = smem_u32(sW + ws * kWStageBytes + nl * 64 + kk * 32);
+          sc = sS[ws * 128 + kk * 64 + nl];
+          dst = smem_u32(sA + as * kAStageBytes + (nl >> 3) * 2048 + kk * 1024 + (nl & 7) * 128);
+          swz = nl & 7;
+        }
+        const uint4 c0 = ld_shared_v4(src);
+        const uint4 c1 = ld_shared_v4(src + 16);
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t w = cw[c];
+          uint32_t o[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t lo = (w >> (8 * h)) & 15u;
+            const uint32_t hi = (w >> (8 * h + 4)) & 15u;
+            o[h] = pack_bf16x2(__fmul_rn(sL[lo], sc), __fmul_rn(sL[hi], sc));
+          }
+          st_shared_v4(dst + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&full_A[as]);
+        mbar_arrive(&empty_W[ws]);
+        if (++as == kStagesA) { as = 0; aph ^= 1u; }
+        if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
+      }
+      if (!ok) break;
+      // LoRA weight-side stages: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
+      for (int ls = 0; ls < p.kb_lora; ++ls) {
+        if (!wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+        const uint32_t abase = smem_u32(sA + as * kAStageBytes);
+        if (MODE == kModeFwd) {
+          // MN-major: K index cr (0..63), M group mg: 64 weight rows of B[c mod r][w0 + 64 mg ..]
+          const int cr = t & 63, mg = t >> 6;
+          const int c = ls * 64 + cr;
+          const uint32_t d = abase + (cr >> 3) * 2048 + mg * 1024 + (cr & 7) * 128;
+          const uint16_t *srcg = p.lora_w + static_cast<int64_t>(c % p.r) * p.lora_ld + w0 + mg * 64;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + ch * 8);
+            st_shared_v4(d + ((ch ^ (cr & 7)) << 4), v.x, v.y, v.z, v.w);
+          }
+        } else {
+          // K-major: row t = input feature k = w0 + t: A[k][c mod r] for c < 2r
+          const uint32_t d = abase + t * 128;
+          const uint16_t *srcg = p.lora_w + static_cast<int64_t>(w0 + t) * p.lora_ld;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int c = ls * 64 + ch * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + (c % p.r));
+            st_shared_v4(d + ((ch ^ (t & 7)) << 4), v.x, v.y, v.z, v.w);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&full_A[as]);
+        if (++as == kStagesA) { as = 0; aph ^= 1u; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace qlora

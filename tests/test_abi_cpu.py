@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI: the library builds/loads on a machine without a
+GPU, exports every function the header declares, and its host-only logic
+(level table, byte sizes, argument validation) agrees with the oracle.  No
+compute call reaches a GPU here."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from bit_nf4_quantized_19_b200 import _abi, build
+from oracle import nf4 as onf4
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _abi.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _abi.header_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _abi.SIGNATURES, f"binding lacks {n}"
+    assert set(_abi.SIGNATURES) == set(names)
+
+
+def test_version_and_status_strings(L):
+    assert L.qlora_version() >= 100
+    for code in range(9):
+        s = L.qlora_status_string(code)
+        assert s and s != b"unknown status"
+    assert L.qlora_status_string(99) == b"unknown status"
+
+
+def test_level_table_bit_identical_to_oracle(L):
+    """The library builds its table with its own inverse-CDF code (Newton on
+    erfc); the oracle uses scipy's ndtri.  Both must give the same fp32 bits."""
+    buf = (ctypes.c_float * 16)()
+    L.qlora_nf4_levels(buf)
+    lib_levels = np.frombuffer(buf, dtype=np.float32).copy()
+    assert np.array_equal(lib_levels.view(np.uint32), onf4.nf4_levels().view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1), (1, 7), (3, 21), (64, 64), (1024, 1024),
+                                       (4096, 4096), (11008, 4096), (1, 1_000_000_000)])
+def test_nf4_bytes_match_oracle(L, rows, cols):
+    c, q, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    tot = L.qlora_nf4_bytes(rows, cols, ctypes.byref(c), ctypes.byref(q), ctypes.byref(s))
+    assert (c.value, q.value, s.value) == onf4.storage_bytes(rows * cols)
+    assert tot == c.value + q.value + s.value
+
+
+def test_bits_per_value_closed_form(L):
+    n = 4096 * 4096
+    tot = L.qlora_nf4_bytes(4096, 4096, None, None, None)
+    assert tot == 8_388_608 + 262_144 + 4_096
+    assert 8.0 * tot / n == 4.126953125
+
+
+def test_argument_errors_before_any_launch(L):
+    null = _abi.NF4Struct(0, 0, 0, 4, 4)
+    assert L.qlora_nf4_quantize(None, 4, 4, ctypes.byref(null), None) == 1
+    assert L.qlora_nf4_dequant(ctypes.byref(null), ctypes.c_void_p(16), None) == 1
+    bad = _abi.NF4Struct(16, 18, 32, 128, 128)            # q8 pointer misaligned
+    assert L.qlora_nf4_dequant(ctypes.byref(bad), ctypes.c_void_p(64), None) == 2
+    ok = _abi.NF4Struct(16, 32, 48, 128, 128)
+    # r out of range / not a multiple of 8
+    for r in (0, 4, 12, 136):
+        assert L.qlora_linear_fwd(ctypes.c_void_p(16), 4, ctypes.byref(ok), ctypes.c_void_p(16),
+                                  ctypes.c_void_p(16), r, 1.0, ctypes.c_void_p(16), None,
+                                  ctypes.c_void_p(16), 1 << 20, None) == 1
+    # shapes the fused GEMM does not cover
+    odd = _abi.NF4Struct(16, 32, 48, 100, 128)
+    assert L.qlora_linear_fwd(ctypes.c_void_p(16), 4, ctypes.byref(odd), ctypes.c_void_p(16),
+                              ctypes.c_void_p(16), 8, 1.0, ctypes.c_void_p(16), None,
+                              ctypes.c_void_p(16), 1 << 20, None) == 3
+    # misaligned activation pointer
+    assert L.qlora_linear_fwd(ctypes.c_void_p(18), 4, ctypes.byref(ok), ctypes.c_void_p(16),
+                              ctypes.c_void_p(16), 8, 1.0, ctypes.c_void_p(16), None,
+                              ctypes.c_void_p(16), 1 << 20, None) == 2
+    assert L.qlora_linear_bwd(None, ctypes.c_void_p(16), None, 4, ctypes.byref(ok),
+                              ctypes.c_void_p(16), ctypes.c_void_p(16), 8, 1.0, None,
+                              ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                              1 << 20, None) == 1
+    assert L.qlora_selftest_wait_timeout(0, None) == 1
+    flags = ctypes.c_uint32()
+    assert L.qlora_get_device_status(None, None) == 1
+
+
+def test_wait_limit_setter_roundtrip(L):
+    old = L.qlora_set_wait_limit_us(123)
+    assert L.qlora_set_wait_limit_us(old) == 123

@@ -109,3 +109,14 @@ def test_rel_fro():
     a = np.ones((3, 3))
     assert linear.rel_fro(a, a) == 0.0
     assert abs(linear.rel_fro(a * 1.001, a) - 1e-3) < 1e-12
+
+
+def test_lora_products_match_full_backward():
+    X, W, A, B, dY = _tiny(4)
+    s = 1.25
+    lp = linear.lora_products(dY, X, A, B, s)
+    g = linear.backward(dY, X, W, A, B, s)
+    _, XA = linear.forward(X, W, A, B, s)
+    np.testing.assert_allclose(lp["XA"], XA, rtol=1e-14, atol=1e-14)
+    for k in ("G", "dA", "dB"):
+        np.testing.assert_allclose(lp[k], g[k], rtol=1e-13, atol=1e-13)
