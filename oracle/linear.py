@@ -45,6 +45,15 @@ def backward(dY, X, Wd, A, B, s: float, XA=None):
     return dict(G=G, dX=dX, dA=dA, dB=dB)
 
 
+def lora_products(dY, X, A, B, s: float):
+    """The rank-r quantities that need no W: XA = X A, G = dY B^T,
+    dA = s X^T G, dB = s XA^T dY (fp64)."""
+    dY, X, A, B = (as_f64(t) for t in (dY, X, A, B))
+    XA = X @ A
+    G = dY @ B.T
+    return dict(XA=XA, G=G, dA=s * (X.T @ G), dB=s * (XA.T @ dY))
+
+
 def forward_rows(X, Wd, A, B, s: float, rows):
     """Y restricted to the given token rows (for sampled checks at full size)."""
     rows = np.asarray(rows)
