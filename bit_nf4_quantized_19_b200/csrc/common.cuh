@@ -196,11 +196,71 @@ QDEV uint4 ld_global_nc_v4(const void *p) {
                : "l"(p));
   return v;
 }
+// prmt.b32 in its default mode: result byte i = byte c[4i+2:4i] of {b, a}
+// (a = bytes 0-3, b = bytes 4-7); if c[4i+3] is set, the selected byte's sign
+// bit is replicated over the whole result byte.  Only c[15:0] is used.
+QDEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 QDEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&b);
 }
 QDEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 QDEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+}  // namespace qlora
+
+namespace qlora {
+
+// ------------------------------------------------------------------ in-register NF4 decode
+// One block's 16 dequantized values bf16_RN(RN32(L[c] * scale)) -- exactly the
+// per-element definition -- kept as two 16-byte tables: lo[q] holds the low
+// bytes and hi[q] the high bytes of entries 4q..4q+3.
+struct Nf4Lut {
+  uint32_t lo[4], hi[4];
+};
+
+QDEV void nf4_build_lut(const float (&L)[16], float scale, Nf4Lut &t) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(__fmul_rn(L[2 * i], scale), __fmul_rn(L[2 * i + 1], scale));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420u);
+    t.hi[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531u);
+  }
+}
+
+// Eight 4-bit codes (element 2j in the low nibble of byte j) -> four bf16x2
+// words in element order.  Bits 0-2 of each code select a byte within an
+// 8-entry half table (prmt); bit 3 picks the half via a byte mask made by
+// prmt's sign-replicate mode; the low and high bytes are then interleaved.
+QDEV void nf4_decode8(uint32_t w, const Nf4Lut &t, uint32_t (&o)[4]) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t sel_hi = sel >> 16;
+  const uint32_t ws = w << 4;
+  const uint32_t m0 = prmt(w, ws, 0x9D8Cu);   // codes 0..3: 0xFF where bit 3 is set
+  const uint32_t m1 = prmt(w, ws, 0xBFAEu);   // codes 4..7
+  {
+    const uint32_t la = prmt(t.lo[0], t.lo[1], sel), lb = prmt(t.lo[2], t.lo[3], sel);
+    const uint32_t ha = prmt(t.hi[0], t.hi[1], sel), hb = prmt(t.hi[2], t.hi[3], sel);
+    const uint32_t lo = (lb & m0) | (la & ~m0);
+    const uint32_t hi = (hb & m0) | (ha & ~m0);
+    o[0] = prmt(lo, hi, 0x5140u);
+    o[1] = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t la = prmt(t.lo[0], t.lo[1], sel_hi), lb = prmt(t.lo[2], t.lo[3], sel_hi);
+    const uint32_t ha = prmt(t.hi[0], t.hi[1], sel_hi), hb = prmt(t.hi[2], t.hi[3], sel_hi);
+    const uint32_t lo = (lb & m1) | (la & ~m1);
+    const uint32_t hi = (hb & m1) | (ha & ~m1);
+    o[2] = prmt(lo, hi, 0x5140u);
+    o[3] = prmt(lo, hi, 0x7362u);
+  }
+}
 
 }  // namespace qlora

@@ -14,25 +14,28 @@
 // and the weight side repeats B^T (or A) twice, so the adapter term is
 // accumulated to ~2^-16 relative precision, not bf16 precision.
 //
-// Warp roles (384 threads, one CTA per SM, persistent over tiles):
+// Warp roles (512 threads, one CTA per SM, persistent over tiles):
 //   warp 0        TMA producer: activation tiles (X / dY, or the LoRA hi/lo
 //                 operand) and packed 4-bit weight tiles + block constants.
 //   warp 1        TMEM allocator and single-thread MMA issuer.
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
-//   warps 8..11   dequant producers: packed codes + constant -> bf16 tile in
-//                 the 128-byte-swizzled UMMA layout, then LoRA weight tiles.
+//   warps 8..15   dequant producers, two warpgroups taking alternate stages:
+//                 packed codes + block constant -> bf16 tile in the
+//                 128-byte-swizzled UMMA layout (one 64-value block per
+//                 thread, decoded through a 16-entry table held in registers),
+//                 then the LoRA weight tiles.
 // Every wait is bounded (see Waiter); a wait that runs out aborts the block.
 #pragma once
 #include "common.cuh"
 
 namespace qlora {
 
-constexpr int kGemmThreads = 384;
+constexpr int kGemmThreads = 512;
 constexpr int kBN = 256;                  // tokens per tile (MMA N)
 constexpr int kWT = 128;                  // weight-side rows per tile (MMA M)
 constexpr int kBK = 64;                   // contraction per stage (one quant block)
 constexpr int kStagesB = 4;               // activation ring
-constexpr int kStagesA = 3;               // dequantized weight ring
+constexpr int kStagesA = 4;               // dequantized weight ring
 constexpr int kStagesW = 4;               // packed code ring
 constexpr int kBStageBytes = kBN * 128;   // 32 KB
 constexpr int kAStageBytes = kWT * 128;   // 16 KB
@@ -253,86 +256,90 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequant producers
-    const int t = tid - 256;            // 0..127
-    int as = 0, ws = 0;
-    uint32_t aph = 0, wph = 0;
+    const int t = (tid - 256) & 127;    // row slot within the stage
+    const int grp = (tid - 256) >> 7;   // warpgroup 0 takes even stages, 1 odd
+    float L[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) L[i] = sL[i];
+    uint32_t a_cnt = 0, w_cnt = 0;      // stages seen so far (all / main only)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int w0 = (tile % p.num_w_tiles) * kWT;
-      for (int kb = 0; kb < p.kb_main; ++kb) {
-        if (!wait_bar(&full_W[ws], wph, wt) || !wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
-        // Which block this thread expands and where its 128-byte row goes.
-        uint32_t src, dst;
-        int swz;
-        float sc;
-        if (MODE == kModeFwd) {
-          // row t of the tile: weight row w0+t, 64 values of K (one block)
-          src = smem_u32(sW + ws * kWStageBytes + t * 32);
-          sc = sS[ws * 128 + t];
-          dst = smem_u32(sA + as * kAStageBytes + t * 128);
-          swz = t & 7;
+      for (int kb = 0; kb < nkb; ++kb, ++a_cnt) {
+        const bool main = kb < p.kb_main;
+        const uint32_t my_w = w_cnt;
+        if (main) ++w_cnt;
+        if ((a_cnt & 1u) != static_cast<uint32_t>(grp)) continue;
+        const int as = static_cast<int>(a_cnt % kStagesA);
+        const uint32_t aph = (a_cnt / kStagesA) & 1u;
+        if (main) {
+          const int ws = static_cast<int>(my_w % kStagesW);
+          const uint32_t wph = (my_w / kStagesW) & 1u;
+          if (!wait_bar(&full_W[ws], wph, wt) || !wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+          uint32_t src, dst;
+          int swz;
+          float sc;
+          if (MODE == kModeFwd) {
+            // row t of the tile: weight row w0+t, 64 values of K (one block), K-major
+            src = smem_u32(sW + ws * kWStageBytes + t * 32);
+            sc = sS[ws * 128 + t];
+            dst = smem_u32(sA + as * kAStageBytes + t * 128);
+            swz = t & 7;
+          } else {
+            // weight row n = kb*64 + nl, 64 values of K from w0 + 64*kk; MN-major:
+            // K index nl, M group kk
+            const int nl = t & 63, kk = t >> 6;
+            src = smem_u32(sW + ws * kWStageBytes + nl * 64 + kk * 32);
+            sc = sS[ws * 128 + kk * 64 + nl];
+            dst = smem_u32(sA + as * kAStageBytes + (nl >> 3) * 2048 + kk * 1024 + (nl & 7) * 128);
+            swz = nl & 7;
+          }
+          const uint4 c0 = ld_shared_v4(src);
+          const uint4 c1 = ld_shared_v4(src + 16);
+          mbar_arrive(&empty_W[ws]);        // codes are in registers now
+          Nf4Lut lut;
+          nf4_build_lut(L, sc, lut);
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+            nf4_decode8(cw[c], lut, o);
+            st_shared_v4(dst + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&full_A[as]);
         } else {
-          // weight row n = kb*64 + nl, 64 values of K starting at w0 + 64*kk;
-          // MN-major: K index nl, M group kk
-          const int nl = t & 63, kk = t >> 6;
-          src = smem_u32(sW + ws * kWStageBytes + nl * 64 + kk * 32);
-          sc = sS[ws * 128 + kk * 64 + nl];
-          dst = smem_u32(sA + as * kAStageBytes + (nl >> 3) * 2048 + kk * 1024 + (nl & 7) * 128);
-          swz = nl & 7;
-        }
-        const uint4 c0 = ld_shared_v4(src);
-        const uint4 c1 = ld_shared_v4(src + 16);
-        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          // LoRA weight-side stage: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
+          const int ls = kb - p.kb_main;
+          if (!wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+          const uint32_t abase = smem_u32(sA + as * kAStageBytes);
+          if (MODE == kModeFwd) {
+            // MN-major: K index cr (0..63), M group mg: B[c mod r][w0 + 64 mg ..]
+            const int cr = t & 63, mg = t >> 6;
+            const int c = ls * 64 + cr;
+            const uint32_t d = abase + (cr >> 3) * 2048 + mg * 1024 + (cr & 7) * 128;
+            const uint16_t *srcg = p.lora_w + static_cast<int64_t>(c % p.r) * p.lora_ld + w0 + mg * 64;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t w = cw[c];
-          uint32_t o[4];
+            for (int ch = 0; ch < 8; ++ch) {
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + ch * 8);
+              st_shared_v4(d + ((ch ^ (cr & 7)) << 4), v.x, v.y, v.z, v.w);
+            }
+          } else {
+            // K-major: row t = input feature k = w0 + t: A[k][c mod r] for c < 2r
+            const uint32_t d = abase + t * 128;
+            const uint16_t *srcg = p.lora_w + static_cast<int64_t>(w0 + t) * p.lora_ld;
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const uint32_t lo = (w >> (8 * h)) & 15u;
-            const uint32_t hi = (w >> (8 * h + 4)) & 15u;
-            o[h] = pack_bf16x2(__fmul_rn(sL[lo], sc), __fmul_rn(sL[hi], sc));
+            for (int ch = 0; ch < 8; ++ch) {
+              const int c = ls * 64 + ch * 8;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + (c % p.r));
+              st_shared_v4(d + ((ch ^ (t & 7)) << 4), v.x, v.y, v.z, v.w);
+            }
           }
-          st_shared_v4(dst + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          fence_proxy_async_smem();
+          mbar_arrive(&full_A[as]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&full_A[as]);
-        mbar_arrive(&empty_W[ws]);
-        if (++as == kStagesA) { as = 0; aph ^= 1u; }
-        if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
-      }
-      if (!ok) break;
-      // LoRA weight-side stages: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
-      for (int ls = 0; ls < p.kb_lora; ++ls) {
-        if (!wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
-        const uint32_t abase = smem_u32(sA + as * kAStageBytes);
-        if (MODE == kModeFwd) {
-          // MN-major: K index cr (0..63), M group mg: 64 weight rows of B[c mod r][w0 + 64 mg ..]
-          const int cr = t & 63, mg = t >> 6;
-          const int c = ls * 64 + cr;
-          const uint32_t d = abase + (cr >> 3) * 2048 + mg * 1024 + (cr & 7) * 128;
-          const uint16_t *srcg = p.lora_w + static_cast<int64_t>(c % p.r) * p.lora_ld + w0 + mg * 64;
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + ch * 8);
-            st_shared_v4(d + ((ch ^ (cr & 7)) << 4), v.x, v.y, v.z, v.w);
-          }
-        } else {
-          // K-major: row t = input feature k = w0 + t: A[k][c mod r] for c < 2r
-          const uint32_t d = abase + t * 128;
-          const uint16_t *srcg = p.lora_w + static_cast<int64_t>(w0 + t) * p.lora_ld;
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int c = ls * 64 + ch * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (c < 2 * p.r) v = *reinterpret_cast<const uint4 *>(srcg + (c % p.r));
-            st_shared_v4(d + ((ch ^ (t & 7)) << 4), v.x, v.y, v.z, v.w);
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&full_A[as]);
-        if (++as == kStagesA) { as = 0; aph ^= 1u; }
       }
     }
   }

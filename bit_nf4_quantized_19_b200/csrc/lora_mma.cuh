@@ -1,0 +1,254 @@
+// Rank-r contractions of the QLoRA adapter on tcgen05 ("QLoRA",
+// ozercemkelahmet.com, How it works, Steps 4-6):
+//   projections   XA = X A,  G = dY B^T              (rows = tokens)
+//   gradients     dA = X^T (sG),  dB = dY^T (sXA)     (rows = input/output features)
+// Every one is a tall-skinny product  D[rows, nn] = Act[rows, c] * Q[nn, c]^T
+// with nn = r (rounded up to 16) or 2r (bf16 hi|lo halves of an fp32
+// operand), so it is bound by reading the bf16 activation (X or dY) once.
+//
+// One CTA computes a 128-row tile over one split of the contraction and writes
+// an fp32 partial tile; a separate reduction sums the splits in a fixed order
+// (deterministic).  The activation side is the MMA's A operand:
+//   K-major  (projections): Act = X / dY tile [128 tokens x 64 c], TMA box {64, 128}
+//   MN-major (gradients):   Act^T tile [128 features x 64 tokens] from X / dY
+//                           [tokens, features]: two TMA boxes {64 features, 64 tokens}
+// Q is always K-major [nn rows x 64 c], TMA box {64, nn}.
+// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 4..7 epilogue.
+#pragma once
+#include "common.cuh"
+
+namespace qlora {
+
+constexpr int kLmThreads = 256;
+constexpr int kLmRows = 128;
+constexpr int kLmABytes = kLmRows * 128;   // 16 KB per stage
+
+struct LoraMmaParams {
+  int rows;              // output rows (tokens for projections, features for gradients)
+  int nn;                // MMA N: multiple of 16, <= 256
+  int stages_total;      // contraction stages of 64
+  int stages_per_split;
+  int num_stages;        // smem ring depth
+  uint32_t tmem_cols;    // power of two >= max(32, nn)
+  float *partial;        // [splits][rows][nn]
+  uint64_t limit_ns;
+};
+
+inline int lora_mma_smem_bytes(int nn, int stages) {
+  return 1024 + stages * (kLmABytes + nn * 128) + 256;
+}
+
+template <bool A_MN>
+__global__ void __launch_bounds__(kLmThreads, 1)
+    lora_mma_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ LoraMmaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int S = p.num_stages;
+  const int b_bytes = p.nn * 128;
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + S * kLmABytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sB + S * b_bytes);
+  uint64_t *empty = full + S;
+  uint64_t *done = empty + S;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = blockIdx.x * kLmRows;
+  const int split = blockIdx.y;
+  const int st0 = split * p.stages_per_split;
+  const int st1 = min(p.stages_total, st0 + p.stages_per_split);
+  const int nst = st1 - st0;
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const Waiter wt{abort_flag, p.limit_ns};
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_act);
+    prefetch_tmap(&tm_q);
+    uint32_t armed = 0, last = 0;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nst; ++i) {
+      if (!wait_bar(&empty[s], ph ^ 1u, wt)) break;
+      const int c0 = (st0 + i) * 64;
+      mbar_arrive_expect_tx(&full[s], kLmABytes + b_bytes);
+      if (A_MN) {
+        tma_load_2d(sA + s * kLmABytes, &tm_act, &full[s], row0, c0);
+        tma_load_2d(sA + s * kLmABytes + 8192, &tm_act, &full[s], row0 + 64, c0);
+      } else {
+        tma_load_2d(sA + s * kLmABytes, &tm_act, &full[s], c0, row0);
+      }
+      tma_load_2d(sB + s * b_bytes, &tm_q, &full[s], c0, 0);
+      armed |= 1u << s;
+      last = (last & ~(1u << s)) | (ph << s);
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    volatile int no_abort = 0;
+    const Waiter fw{&no_abort, p.limit_ns};
+    for (int k = 0; k < S; ++k)
+      if (armed & (1u << k)) wait_bar(&full[k], (last >> k) & 1u, fw);
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = make_idesc_bf16(kLmRows, p.nn, A_MN, false);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = 0; i < nst; ++i) {
+      if (!wait_bar(&full[s], ph, wt)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a = smem_u32(sA + s * kLmABytes);
+      const uint32_t b = smem_u32(sB + s * b_bytes);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = A_MN ? sw128_desc(a + k * 2048, 8192, 1024) : sw128_desc(a + k * 32, 16, 1024);
+        const uint64_t bd = sw128_desc(b + k * 32, 16, 1024);
+        mma_bf16_ss(tmem_base, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+      }
+      mma_commit(&empty[s]);
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    (void)ok;
+    mma_commit(done);   // also drains every issued MMA before TMEM is released
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const int row = row0 + q * 32 + lane;
+    volatile int no_abort = 0;
+    const Waiter dw{&no_abort, p.limit_ns};
+    const bool got = __all_sync(0xffffffffu, wait_bar(done, 0, dw) ? 1 : 0);
+    tc_fence_after();
+    float *dst = p.partial + (static_cast<int64_t>(split) * p.rows + row) * p.nn;
+    for (int c = 0; c < p.nn; c += 16) {
+      uint32_t v[16];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+            "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+            "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+          : "r"(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c)));
+      tmem_wait_ld();
+      if (row < p.rows) {
+        float4 *d4 = reinterpret_cast<float4 *>(dst + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float4 o;
+          if (got && nst > 0) {
+            o = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          } else {
+            o = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          d4[j] = o;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------- helpers around it
+// AT[j][k] = A[k][j]: the adapter A [K, r] as the K-major operand [r, K].
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__restrict__ A, int K,
+                                                             int r, uint16_t *__restrict__ AT) {
+  const int64_t total = static_cast<int64_t>(K) * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = i / K, k = i - j * K;
+    AT[i] = A[k * r + j];
+  }
+}
+
+QDEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+  hi = *reinterpret_cast<const uint16_t *>(&h);
+  lo = *reinterpret_cast<const uint16_t *>(&l);
+}
+
+// Projection reduction: out[m][j] = sum over splits (in order) of partial[sp][m][j];
+// then s*out split into bf16 hi/lo, written as hl [M, 2r] (hi in columns 0..r-1,
+// lo in r..2r-1) and/or hlT [2r, ldT].  Thread index runs over (j, m) with m fastest.
+__global__ void __launch_bounds__(256) proj_reduce_kernel(const float *__restrict__ partial, int splits,
+                                                          int M, int nn, int r, float s,
+                                                          float *__restrict__ out,
+                                                          uint16_t *__restrict__ hl,
+                                                          uint16_t *__restrict__ hlT, int ldT) {
+  const int64_t total = static_cast<int64_t>(M) * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(i / M);
+    const int m = static_cast<int>(i - static_cast<int64_t>(j) * M);
+    float v = 0.f;
+    for (int sp = 0; sp < splits; ++sp) v += partial[(static_cast<int64_t>(sp) * M + m) * nn + j];
+    if (out) out[static_cast<int64_t>(m) * r + j] = v;
+    uint16_t h, l;
+    split_hilo(s * v, h, l);
+    if (hl) {
+      hl[static_cast<int64_t>(m) * 2 * r + j] = h;
+      hl[static_cast<int64_t>(m) * 2 * r + r + j] = l;
+    }
+    if (hlT) {
+      hlT[static_cast<int64_t>(j) * ldT + m] = h;
+      hlT[static_cast<int64_t>(r + j) * ldT + m] = l;
+    }
+  }
+}
+
+// hlT [2r, ldT] = hi/lo of s*v for an fp32 v [M, r] (the saved XA in the backward).
+__global__ void __launch_bounds__(256) hilo_t_kernel(const float *__restrict__ v, int M, int r, float s,
+                                                     uint16_t *__restrict__ hlT, int ldT) {
+  const int64_t total = static_cast<int64_t>(M) * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(i / M);
+    const int m = static_cast<int>(i - static_cast<int64_t>(j) * M);
+    uint16_t h, l;
+    split_hilo(s * v[static_cast<int64_t>(m) * r + j], h, l);
+    hlT[static_cast<int64_t>(j) * ldT + m] = h;
+    hlT[static_cast<int64_t>(r + j) * ldT + m] = l;
+  }
+}
+
+// Gradient reduction: g[c][j] = sum over splits of (partial[sp][c][j] + partial[sp][c][r+j])
+// (hi and lo halves).  layout 0 writes out[c][j] (dA [K, r]); layout 1 out[j][c] (dB [r, N]).
+__global__ void __launch_bounds__(256) grad_reduce_hilo_kernel(const float *__restrict__ partial,
+                                                               int splits, int C, int r, int layout,
+                                                               float *__restrict__ out) {
+  const int64_t total = static_cast<int64_t>(C) * r;
+  const int nn = 2 * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t c, j;
+    if (layout == 0) { c = i / r; j = i - c * r; }
+    else { j = i / C; c = i - j * C; }
+    float v = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float *pp = partial + (static_cast<int64_t>(sp) * C + c) * nn;
+      v += pp[j] + pp[r + j];
+    }
+    out[i] = v;
+  }
+}
+
+}  // namespace qlora

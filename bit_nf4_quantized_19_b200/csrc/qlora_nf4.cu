@@ -8,7 +8,7 @@
 
 #include "common.cuh"
 #include "gemm_kernel.cuh"
-#include "lora_kernels.cuh"
+#include "lora_mma.cuh"
 #include "nf4_table.hpp"
 #include "quant_kernels.cuh"
 
@@ -156,19 +156,50 @@ struct Workspace {
   }
 };
 
-int grad_splits(int64_t M, int64_t C, int sms) {
-  const int64_t ctiles = (C + kGradCT - 1) / kGradCT;
-  int64_t splits = (2 * static_cast<int64_t>(sms) + ctiles - 1) / ctiles;
-  const int64_t maxs = (M + kGradTM - 1) / kGradTM;
-  if (splits > maxs) splits = maxs;
-  if (splits < 1) splits = 1;
-  if (splits > 64) splits = 64;
-  return static_cast<int>(splits);
+// ---- launch geometry of the rank-r contractions (lora_mma_kernel)
+struct LmGeom {
+  int nn, row_tiles, stages_total, sps, splits, num_stages;
+  uint32_t tmem_cols;
+  size_t partial_bytes;
+};
+
+LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
+  LmGeom g{};
+  g.nn = nn;
+  g.row_tiles = static_cast<int>((rows + kLmRows - 1) / kLmRows);
+  g.stages_total = static_cast<int>((contraction + 63) / 64);
+  int want = (2 * sms + g.row_tiles - 1) / g.row_tiles;
+  if (want < 1) want = 1;
+  if (want > g.stages_total) want = g.stages_total;
+  g.sps = (g.stages_total + want - 1) / want;
+  g.splits = (g.stages_total + g.sps - 1) / g.sps;
+  int st = (110 * 1024) / (kLmABytes + nn * 128);
+  g.num_stages = st < 2 ? 2 : (st > 8 ? 8 : st);
+  uint32_t tc = 32;
+  while (tc < static_cast<uint32_t>(nn)) tc <<= 1;
+  g.tmem_cols = tc;
+  g.partial_bytes = static_cast<size_t>(g.splits) * static_cast<size_t>(rows) * nn * 4;
+  return g;
 }
 
-size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r) {
+int nn_proj(int r) { return (r + 15) / 16 * 16; }
+int64_t pad8(int64_t m) { return (m + 7) / 8 * 8; }
+
+size_t partial_max(int64_t M, int64_t N, int64_t K, int r, int sms) {
+  size_t a = lm_geom(M, K, nn_proj(r), sms).partial_bytes;
+  size_t b = lm_geom(M, N, nn_proj(r), sms).partial_bytes;
+  size_t c = lm_geom(K, M, 2 * r, sms).partial_bytes;
+  size_t d = lm_geom(N, M, 2 * r, sms).partial_bytes;
+  size_t x = a > b ? a : b;
+  size_t y = c > d ? c : d;
+  return x > y ? x : y;
+}
+
+size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
-  b += align256(static_cast<size_t>(N) * (K / 64) * 4);        // expanded constants
+  b += align256(static_cast<size_t>(N) * (K / 64) * 4);        // expanded block constants
+  b += align256(static_cast<size_t>(r) * K * 2);               // A^T
+  b += align256(partial_max(M, N, K, r, sms));                 // split partials
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*XA hi/lo
   b += align256(static_cast<size_t>(M) * r * 4);               // XA when XA_out is NULL
   return b + 256;
@@ -177,12 +208,13 @@ size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r) {
 size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
   b += align256(static_cast<size_t>(N) * (K / 64) * 4);
+  b += align256(static_cast<size_t>(r) * K * 2);               // A^T (XA recompute)
+  b += align256(partial_max(M, N, K, r, sms));
   b += align256(static_cast<size_t>(M) * r * 4);               // G
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*G hi/lo
+  b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*G hi/lo transposed
+  b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*XA hi/lo transposed
   b += align256(static_cast<size_t>(M) * r * 4);               // XA recomputed
-  b += align256(static_cast<size_t>(M) * 2 * r * 2);           // its hi/lo (unused output)
-  b += align256(static_cast<size_t>(grad_splits(M, K, sms)) * K * r * 4);
-  b += align256(static_cast<size_t>(grad_splits(M, N, sms)) * N * r * 4);
   return b + 256;
 }
 
@@ -211,33 +243,88 @@ qlora_status launch_expand_scales(const qlora_nf4_t *Wq, float *S, cudaStream_t 
   return cuda_status(cudaGetLastError());
 }
 
-qlora_status launch_project(const uint16_t *P, int64_t M, int64_t C, const uint16_t *Q,
-                            bool q_rows_are_c, int r, float s, float *out, uint16_t *hl,
-                            cudaStream_t st) {
-  const int grid = static_cast<int>((M + kProjTM - 1) / kProjTM);
-  const size_t smem = (kProjTM * (kProjKC + 1) + kProjKC * r) * sizeof(float);
-  LaunchTimer lt(QLORA_K_PROJECT, st);
-  lora_project_kernel<<<grid, kProjThreads, smem, st>>>(P, static_cast<int>(M), static_cast<int>(C),
-                                                        Q, q_rows_are_c ? 1 : 0, r, s, out, hl);
+int grid_for(int64_t total, int sms) {
+  int64_t g = (total + 255) / 256;
+  if (g > static_cast<int64_t>(sms) * 8) g = static_cast<int64_t>(sms) * 8;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
+// D[rows, nn] partials = act (K-major rows x c, or MN-major c x rows) * q^T, over splits.
+template <bool A_MN>
+qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_cols,
+                             const uint16_t *qop, int64_t q_rows, int64_t q_cols, int64_t q_pitch,
+                             int64_t rows, int64_t contraction, int nn, float *partial, int sms,
+                             cudaStream_t st, LmGeom *geom_out) {
+  const LmGeom g = lm_geom(rows, contraction, nn, sms);
+  CUtensorMap tm_act, tm_q;
+  // act is [act_rows (tokens), act_cols (features)] row-major bf16
+  if (!make_map_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, act_cols, act_rows, act_cols * 2,
+                   64, A_MN ? 64 : kLmRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  if (!make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qop, q_cols, q_rows, q_pitch * 2, 64,
+                   static_cast<uint32_t>(nn), CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  LoraMmaParams p{};
+  p.rows = static_cast<int>(rows);
+  p.nn = nn;
+  p.stages_total = g.stages_total;
+  p.stages_per_split = g.sps;
+  p.num_stages = g.num_stages;
+  p.tmem_cols = g.tmem_cols;
+  p.partial = partial;
+  p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
+  const int smem = lora_mma_smem_bytes(nn, g.num_stages);
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[A_MN ? 1 : 0]) {
+    if (cudaFuncSetAttribute(lora_mma_kernel<A_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    attr_set[A_MN ? 1 : 0] = true;
+  }
+  dim3 grid(static_cast<unsigned>(g.row_tiles), static_cast<unsigned>(g.splits));
+  LaunchTimer lt(A_MN ? QLORA_K_GRAD : QLORA_K_PROJECT, st);
+  lora_mma_kernel<A_MN><<<grid, kLmThreads, smem, st>>>(tm_act, tm_q, p);
+  if (geom_out) *geom_out = g;
   return cuda_status(cudaGetLastError());
 }
 
-qlora_status launch_grad(const uint16_t *P, const float *F, int64_t M, int64_t C, int r, float s,
-                         int layout, float *out, float *part, int sms, cudaStream_t st) {
-  const int splits = grad_splits(M, C, sms);
-  const int tps = static_cast<int>(((M + splits - 1) / splits + kGradTM - 1) / kGradTM * kGradTM);
-  dim3 grid(static_cast<unsigned>((C + kGradCT - 1) / kGradCT), static_cast<unsigned>(splits));
-  const size_t smem = (kGradTM * kGradCT + kGradTM * r) * sizeof(float);
-  {
-    LaunchTimer lt(QLORA_K_GRAD, st);
-    lora_grad_partial_kernel<<<grid, kGradThreads, smem, st>>>(P, F, static_cast<int>(M),
-                                                               static_cast<int>(C), r, tps, part);
-  }
-  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
-  int rgrid = static_cast<int>((C * r + 255) / 256);
-  if (rgrid > sms * 8) rgrid = sms * 8;
+// XA = X A (or G = dY B^T): fp32 [M, r] plus hi/lo of s*result in [M, 2r] and/or [2r, pad8(M)].
+qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const uint16_t *qT,
+                               int r, float s, float *out, uint16_t *hl, uint16_t *hlT,
+                               float *partial, int sms, cudaStream_t st) {
+  LmGeom g;
+  qlora_status e = launch_lora_mma<false>(act, M, C, qT, r, C, C, M, C, nn_proj(r), partial, sms, st, &g);
+  if (e != QLORA_OK) return e;
   LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
-  lora_grad_reduce_kernel<<<rgrid, 256, 0, st>>>(part, splits, static_cast<int>(C), r, s, layout, out);
+  proj_reduce_kernel<<<grid_for(M * r, sms), 256, 0, st>>>(partial, g.splits, static_cast<int>(M), g.nn,
+                                                           r, s, out, hl, hlT, static_cast<int>(pad8(M)));
+  return cuda_status(cudaGetLastError());
+}
+
+qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *hlT, int sms,
+                           cudaStream_t st) {
+  LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
+  hilo_t_kernel<<<grid_for(M * r, sms), 256, 0, st>>>(v, static_cast<int>(M), r, s, hlT,
+                                                       static_cast<int>(pad8(M)));
+  return cuda_status(cudaGetLastError());
+}
+
+// g = act^T * (hi + lo) over tokens: act [M, C] bf16, hlT [2r, pad8(M)]; out dA [C, r] or dB [r, C].
+qlora_status launch_grad(const uint16_t *act, int64_t M, int64_t C, const uint16_t *hlT, int r,
+                         int layout, float *out, float *partial, int sms, cudaStream_t st) {
+  LmGeom g;
+  qlora_status e = launch_lora_mma<true>(act, M, C, hlT, 2 * r, M, pad8(M), C, M, 2 * r, partial, sms,
+                                         st, &g);
+  if (e != QLORA_OK) return e;
+  LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
+  grad_reduce_hilo_kernel<<<grid_for(C * r, sms), 256, 0, st>>>(partial, g.splits, static_cast<int>(C), r,
+                                                                layout, out);
+  return cuda_status(cudaGetLastError());
+}
+
+qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT, int sms, cudaStream_t st) {
+  LaunchTimer lt(QLORA_K_EXPAND, st);
+  transpose_bf16_kernel<<<grid_for(K * r, sms), 256, 0, st>>>(A, static_cast<int>(K), r, AT);
   return cuda_status(cudaGetLastError());
 }
 
@@ -384,7 +471,7 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
   int sms = 148;
   DeviceInfo *d = nullptr;
   if (device_info(&d) == QLORA_OK) sms = d->sms;
-  const size_t f = fwd_workspace(M, N, K, r), b = bwd_workspace(M, N, K, r, sms);
+  const size_t f = fwd_workspace(M, N, K, r, sms), b = bwd_workspace(M, N, K, r, sms);
   return f > b ? f : b;
 }
 
@@ -403,14 +490,19 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
   DeviceInfo *d = nullptr;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t N = Wq->rows, K = Wq->cols;
-  if (!workspace || workspace_bytes < fwd_workspace(M, N, K, r)) return QLORA_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < fwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
+  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
+  float *part = static_cast<float *>(ws.take(partial_max(M, N, K, r, d->sms)));
   uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  if (!S || !hl || !xa) return QLORA_ERR_WORKSPACE;
+  if (!S || !AT || !part || !hl || !xa) return QLORA_ERR_WORKSPACE;
+  // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps
+  if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, part, d->sms, stream)) != QLORA_OK)
+    return st;
   if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
-  if ((st = launch_project(X, M, K, A, true, r, s, xa, hl, stream)) != QLORA_OK) return st;
   return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, d->sms, stream);
 }
 
@@ -432,29 +524,33 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
   const int64_t N = Wq->rows, K = Wq->cols;
   if (!workspace || workspace_bytes < bwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
+  const size_t hlT_bytes = static_cast<size_t>(2 * r) * pad8(M) * 2;
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
+  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
+  float *part = static_cast<float *>(ws.take(partial_max(M, N, K, r, d->sms)));
   float *G = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   uint16_t *ghl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
+  uint16_t *ghlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
+  uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  uint16_t *xa_hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
-  float *partA = static_cast<float *>(ws.take(static_cast<size_t>(grad_splits(M, K, d->sms)) * K * r * 4));
-  float *partB = static_cast<float *>(ws.take(static_cast<size_t>(grad_splits(M, N, d->sms)) * N * r * 4));
-  if (!S || !G || !ghl || !xa_ws || !xa_hl || !partA || !partB) return QLORA_ERR_WORKSPACE;
-  const float *xa = XA;
-  if (!xa) {
-    if ((st = launch_project(X, M, K, A, true, r, 1.0f, xa_ws, xa_hl, stream)) != QLORA_OK) return st;
-    xa = xa_ws;
-  }
-  // G = dY B^T (and s*G hi/lo for the fused dX GEMM)
-  if ((st = launch_project(dY, M, N, B, false, r, s, G, ghl, stream)) != QLORA_OK) return st;
-  if (dX) {
-    if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
-    if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, d->sms, stream)) != QLORA_OK)
+  if (!S || !AT || !part || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
+  // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from X and A)
+  if (XA) {
+    if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
+  } else {
+    if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+    if ((st = launch_projection(X, M, K, AT, r, s, xa_ws, nullptr, xahlT, part, d->sms, stream)) != QLORA_OK)
       return st;
   }
-  // dA = s X^T G  [K, r];  dB = s XA^T dY  [r, N]
-  if ((st = launch_grad(X, G, M, K, r, s, 0, dA, partA, d->sms, stream)) != QLORA_OK) return st;
-  return launch_grad(dY, xa, M, N, r, s, 1, dB, partB, d->sms, stream);
+  // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA)
+  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, part, d->sms, stream)) != QLORA_OK) return st;
+  if (dX) {
+    if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
+    if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, d->sms, stream)) != QLORA_OK) return st;
+  }
+  // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
+  if ((st = launch_grad(X, M, K, ghlT, r, 0, dA, part, d->sms, stream)) != QLORA_OK) return st;
+  return launch_grad(dY, M, N, xahlT, r, 1, dB, part, d->sms, stream);
 }
 
 qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags) {

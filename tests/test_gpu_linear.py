@@ -113,3 +113,27 @@ def test_linear_llama7b_shapes_sampled_rows(q, N, K):
     got = _run(q, p)
     rows = np.unique(np.concatenate([[0, 4095], np.random.default_rng(5).integers(0, 4096, 94)]))
     _check(p, got, rows=rows)
+
+
+@pytest.mark.parametrize("N,K", [(256, 384), (384, 256), (128, 1024)])
+def test_gemm_dequant_bit_exact_one_hot(q, N, K):
+    """With X = I (K one-hot tokens) and A = 0 every output of the forward is a
+    single product 1 * w, so Y = deq(W)^T exactly; with dY = I (N tokens),
+    dX = deq(W).  The dequantization inside both fused GEMMs must therefore
+    equal the oracle's dequantized bf16 bit for bit."""
+    import torch
+    from synth import normal_bf16
+    Wb = normal_bf16(0, f"onehot{N}x{K}", (N, K), 0.02)
+    ref = H.oracle_deq_bits(Wb)                                   # [N, K] bf16 bits
+    Wq = q.nf4_quantize(H.bits_to_dev(Wb))
+    r = 16
+    A = torch.zeros(K, r, dtype=torch.bfloat16, device="cuda")
+    B = torch.randn(r, N, device="cuda").to(torch.bfloat16)
+    Xi = torch.eye(K, dtype=torch.bfloat16, device="cuda")
+    Y, _ = q.linear_fwd(Xi, Wq, A, B, 2.0)
+    dYi = torch.eye(N, dtype=torch.bfloat16, device="cuda")
+    X0 = torch.zeros(N, K, dtype=torch.bfloat16, device="cuda")
+    dX, _, _ = q.linear_bwd(dYi, X0, None, Wq, A, B, 2.0)
+    torch.cuda.synchronize()
+    assert np.array_equal(H.dev_to_bits(Y), ref.T)
+    assert np.array_equal(H.dev_to_bits(dX), ref)
