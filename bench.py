@@ -208,7 +208,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-subpaths", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="M,N,K: small profiling case (two fwd+bwd of one projection), no JSON")
     args = ap.parse_args()
+    if args.case:
+        return profile_case(*[int(v) for v in args.case.split(",")])
     args.warmup = max(3, args.warmup)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -239,12 +243,12 @@ def main():
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
+    from bit_nf4_quantized_19_b200.dp import GradBucket
     layers = []
-    grad_numel = sum(K * RANK_R + RANK_R * N for (_, N, K) in SHAPES)
-    flat_grads = torch.zeros(grad_numel, dtype=torch.float32, device=dev)
-    flat_host = torch.empty(grad_numel, dtype=torch.float32).pin_memory()
-    off = 0
-    for p in hp:
+    bucket = GradBucket([(N, K, RANK_R) for (_, N, K) in SHAPES], dev)
+    flat_grads = bucket.flat
+    flat_host = torch.empty(flat_grads.numel(), dtype=torch.float32).pin_memory()
+    for p, (dA, dB) in zip(hp, bucket.views):
         M, N, K, r = p["M"], p["N"], p["K"], p["r"]
         Wq = q.nf4_quantize(to_dev(p["W"]))
         L = dict(M=M, N=N, K=K, r=r, s=p["s"], Wq=Wq, X=to_dev(p["X"]), dY=to_dev(p["dY"]),
@@ -252,10 +256,7 @@ def main():
                  Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
                  XA=torch.empty(M, r, dtype=torch.float32, device=dev),
                  dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
-                 dA=flat_grads[off:off + K * r].view(K, r),
-                 dB=flat_grads[off + K * r:off + K * r + r * N].view(r, N),
-                 ws=q.make_workspace(M, N, K, r, dev))
-        off += K * r + r * N
+                 dA=dA, dB=dB, ws=q.make_workspace(M, N, K, r, dev))
         L["hX"] = torch.from_numpy(np.ascontiguousarray(p["X"]).view(np.int16)).view(torch.bfloat16).pin_memory()
         L["hdY"] = torch.from_numpy(np.ascontiguousarray(p["dY"]).view(np.int16)).view(torch.bfloat16).pin_memory()
         layers.append(L)
@@ -268,8 +269,7 @@ def main():
                          XA=L["XA"])
             q.linear_bwd(L["dY"], L["X"], L["XA"], L["Wq"], L["A"], L["B"], L["s"],
                          workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
-        if world > 1:
-            dist.all_reduce(flat_grads)
+        bucket.allreduce_()       # the one exchange of data-parallel adapter training
 
     flops_per_step_rank = sum(step_flops(M, N, K, RANK_R) for (M, N, K) in SHAPES)
 
@@ -389,6 +389,29 @@ def main():
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def profile_case(M, N, K, r=RANK_R):
+    """Two forward + backward passes of one projection through the public API
+    (seeded device inputs); the case that the ncu captures under profiles/ use."""
+    import torch
+    import bit_nf4_quantized_19_b200 as q
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    W = (torch.randn(N, K, generator=g, device="cuda") * W_STD).to(torch.bfloat16)
+    X = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
+    dY = torch.randn(M, N, generator=g, device="cuda").to(torch.bfloat16)
+    A = (torch.randn(K, r, generator=g, device="cuda") / r).to(torch.bfloat16)
+    B = (torch.randn(r, N, generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+    Wq = q.nf4_quantize(W)
+    ws = q.make_workspace(M, N, K, r, X.device)
+    for _ in range(2):
+        Y, XA = q.linear_fwd(X, Wq, A, B, ALPHA / r, workspace=ws)
+        q.linear_bwd(dY, X, XA, Wq, A, B, ALPHA / r, workspace=ws)
+    torch.cuda.synchronize()
+    code, flags = q.device_status()
+    print("case", M, N, K, "status", code, flags)
+    return 0 if code == 0 else 1
 
 
 def hbm_subpaths(q, torch, dev, stream, P, flush):
