@@ -19,6 +19,8 @@ STATUS = {
     6: "QLORA_ERR_DEVICE_CHECK", 7: "QLORA_ERR_WORKSPACE", 8: "QLORA_ERR_NO_DEVICE",
 }
 QLORA_OK = 0
+QLORA_ERR_WORKSPACE = 7
+NOALLOC_SCRATCH_BYTES = 16 << 20
 QLORA_ERR_TIMEOUT = 5
 DEVSTAT_TIMEOUT = 1
 DEVSTAT_NONFINITE = 2
@@ -58,6 +60,7 @@ SIGNATURES = {
     "qlora_nf4_dequant": (_int, [_nf4p, _vp, _vp]),
     "qlora_linear_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_fwd_noalloc": (_int, [_vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp,
                                 _vp, _sz, _vp]),
     "qlora_get_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),

@@ -623,3 +623,51 @@ extern "C" qlora_status qlora_selftest_wait_timeout(uint32_t timeout_us, qlora_s
   selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
   return cuda_status(cudaGetLastError());
 }
+
+// ------------------------------------------------------------------ forward without a workspace
+// For callers that cannot allocate device memory (a plain host program linking only
+// this library, or a runtime whose device memory is all planned up front): the
+// forward's scratch comes from one file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library holds this array until exit.
+namespace {
+constexpr size_t kNoallocScratchBytes = QLORA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+struct NoallocSlot {
+  bool ready = false;
+  void *ptr = nullptr;
+};
+NoallocSlot g_noalloc_slot[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the array on the current device, looked up once per device
+// (in host code the array's name is only a host-side stand-in, not a device address).
+qlora_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  NoallocSlot &slot = g_noalloc_slot[dev];
+  if (!slot.ready) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
+    slot.ptr = p;
+    slot.ready = true;
+  }
+  *out = slot.ptr;
+  return QLORA_OK;
+}
+}  // namespace
+
+extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
+                                                 const uint16_t *A, const uint16_t *B, int r, float s,
+                                                 uint16_t *Y, float *XA_out, qlora_stream_t stream) {
+  qlora_status st = check_nf4(Wq);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
+  DeviceInfo *d = nullptr;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  if (fwd_workspace(M, Wq->rows, Wq->cols, r, d->sms) > kNoallocScratchBytes) return QLORA_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != QLORA_OK) return st;
+  return qlora_linear_fwd(X, M, Wq, A, B, r, s, Y, XA_out, scratch, kNoallocScratchBytes, stream);
+}

@@ -142,6 +142,34 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
                               size_t workspace_bytes, qlora_stream_t stream);
 
 /*
+ * Forward without a workspace argument, for callers that cannot allocate device
+ * memory: for example a host program that links only this library and has no
+ * device allocator of its own, or a runtime that hands out all device memory
+ * from an arena planned up front and forbids allocations at call time.  (No
+ * counterpart in the paper: this is a packaging variant of qlora_linear_fwd.)
+ *
+ * Computes exactly what qlora_linear_fwd computes, with its scratch space taken
+ * from one array of QLORA_NOALLOC_SCRATCH_BYTES that the library reserves in
+ * device memory of every GPU that loads it (held until the process exits).
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - Returns QLORA_ERR_WORKSPACE, before launching anything, when the call
+ *     needs more scratch than that (the need grows with M, N*K/16 and r;
+ *     4096 tokens on an 11008 x 4096 weight with r = 16 needs about 5 MB).
+ *   - The first call on each device looks up the array's device address with
+ *     cudaGetSymbolAddress while that device is current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one array, so calls whose executions
+ *     overlap on the GPU (different streams, or host threads) race on it and
+ *     corrupt each other's results; serialize them.  No byte of the array needs
+ *     to start at zero: each call writes every scratch byte before reading it.
+ * Other arguments, shapes and errors as qlora_linear_fwd.
+ */
+#define QLORA_NOALLOC_SCRATCH_BYTES (16u << 20)
+qlora_status qlora_linear_fwd_noalloc(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
+                                      const uint16_t *A, const uint16_t *B, int r, float s,
+                                      uint16_t *Y, float *XA_out, qlora_stream_t stream);
+
+/*
  * Backward of the adapted linear layer ([STEPS] Step 6: gradients flow through
  * the dequantized weights into the adapters; W is frozen, no dW):
  *   G  = dY B^T                   (fp32 [M, r], internal)
