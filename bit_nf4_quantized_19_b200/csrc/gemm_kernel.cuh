@@ -1,7 +1,7 @@
 // Dequant-fused tcgen05 GEMM for the QLoRA linear layer (sm_100a).
 //
 // Forward ("QLoRA", ozercemkelahmet.com, How it works, Step 5; essay at
-// fanfani.net, "store in four bits, compute in sixteen"):
+// fanfani.net, section "The crucial split"):
 //     Y^T[n, m] = sum_k deq(W)[n, k] X[m, k]  +  sum_c B'[n, c] XAhl[m, c]
 // dX (Step 6: gradients flow through the dequantized weights):
 //     dX^T[k, m] = sum_n deq(W)[n, k] dY[m, n] +  sum_c A'[k, c] Ghl[m, c]

@@ -9,8 +9,8 @@
  *           How It Works 1-2 and Training Flow.
  *   [STEPS] "QLoRA" (ozercemkelahmet.com/tools/qlora), How it works, Steps 1-6,
  *           and "A worked example".
- *   [SPLIT] "QLoRA" essay (fanfani.net/articles/qlora), "The crucial split: store in
- *           four bits, compute in sixteen" (the display formula W_4bit -> W_16bit -> W_0 + BA).
+ *   [SPLIT] "QLoRA" essay (fanfani.net/articles/qlora), section "The crucial split" and
+ *           its display formula (4-bit W expanded to 16 bits, used in W_0 + BA).
  *
  * Conventions for every entry point
  *   - bf16 tensors are passed as pointers to IEEE bfloat16 bit patterns (uint16_t).
@@ -86,8 +86,8 @@ const char *qlora_status_string(qlora_status s);
  * The 16 NF4 levels the library uses, sorted ascending, in `out[16]` (host
  * memory).  Built on the host from the inverse normal CDF at evenly spaced
  * probabilities in [0.5, (1-1/32 + 1-1/30)/2]: 8 positive levels, 7 negative,
- * one exact zero, normalised to [-1, 1] ([NF4] "levels at quantiles of the
- * normal distribution ... each bin holds equal probability mass").
+ * one exact zero, normalised to [-1, 1] ([NF4]: levels at normal quantiles,
+ * the same probability mass in every bin).
  */
 void qlora_nf4_levels(float out[16]);
 

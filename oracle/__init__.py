@@ -11,8 +11,8 @@ on 32-bit values):
 
 * ``nf4.nf4_levels``  -- the 16 NormalFloat levels.  Sources: "QLoRA"
   (ai360xpert.com), How It Works 1; "QLoRA: Efficient Finetuning of Quantized
-  LLMs" (crackai.dev), How It Works 1 ("levels placed at quantiles of the normal
-  distribution ... each bin holds equal probability mass"); "QLoRA"
+  LLMs" (crackai.dev), How It Works 1 (levels at normal quantiles, the same
+  probability mass in every bin); "QLoRA"
   (ozercemkelahmet.com), How it works -- Why NormalFloat.
 * ``nf4.quantize``    -- blockwise absmax (64 values), nearest level, two codes
   per byte; then the 8-bit double quantization of the block constants in groups
@@ -20,8 +20,7 @@ on 32-bit values):
   works, Steps 1-3 and "A worked example"; crackai.dev, How It Works 2.
 * ``nf4.dequantize``  -- level times reconstructed block constant, rounded to the
   bf16 compute type.  Sources: ozercemkelahmet.com, Overview and Step 5;
-  "QLoRA" essay (fanfani.net), "The crucial split: store in four bits, compute
-  in sixteen".
+  "QLoRA" essay (fanfani.net), section "The crucial split".
 * ``linear.forward`` / ``linear.backward`` -- Y = X deq(W)^T + s (X A) B and its
   gradients for X, A, B (W frozen), accumulated in fp64.  Sources:
   ozercemkelahmet.com, How it works, Steps 5-6.

@@ -13,7 +13,7 @@ GROUP = 256         # first-level constants per second-level constant (reading; 
 ZERO_CODE = 7       # index of the exact-zero level in the sorted table
 
 # Upper quantile of the table construction: the mean of 1 - 1/32 and 1 - 1/30.
-# A named constant (reading); the pages only say "quantiles of a normal distribution".
+# A named constant (reading); the pages only place the levels at normal quantiles.
 P_MAX = 0.5 * ((1.0 - 1.0 / 32.0) + (1.0 - 1.0 / 30.0))
 
 
@@ -150,7 +150,7 @@ def unpack_codes(packed: np.ndarray, n: int) -> np.ndarray:
 def double_quantize(absmax: np.ndarray):
     """8-bit codes for the per-block constants, in groups of 256, with one fp32
     second-level constant per group ("QLoRA", ozercemkelahmet.com, How it works,
-    Step 3; crackai.dev, How It Works 2: "from 32-bit to 8-bit").
+    Step 3; crackai.dev, How It Works 2: constants go from 32 to 8 bits).
 
     Reading: a_b >= 0, so an unsigned linear code over [0, c_g] with
     step_g = RN32(c_g / 255) and q8_b = min(255, rint_even(RN32(a_b / step_g))).

@@ -77,7 +77,7 @@ def test_table_shape_monotone_exact_ends():
 def test_table_denser_near_zero():
     L = nf4.nf4_levels().astype(np.float64)
     gaps = np.diff(L)
-    # spacing grows away from zero on both sides ("more buckets near zero")
+    # spacing grows away from zero on both sides (denser levels near zero)
     assert np.all(np.diff(gaps[7:]) > 0) and np.all(np.diff(gaps[:7]) < 0)
 
 
@@ -133,7 +133,7 @@ def test_worked_example(golden):
     np.testing.assert_allclose(xn, g["normalised"], rtol=0, atol=1e-7)
     L = nf4.nf4_levels()
     lv = L[q["codes_unpacked"]]
-    # step 2 is only "supposed" on the page: three of the four agree with the
+    # step 2 is a hypothetical on the page: three of the four agree with the
     # NF4 levels to 0.02; for 0.125 the nearest NF4 level is 0.1609, not 0.1.
     sup = np.array(g["supposed"])
     assert np.all(np.abs(lv[1:] - sup[1:]) < 0.02)
