@@ -112,14 +112,15 @@ QDEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" 
 QDEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulator.
+// No "memory" clobber: the operands are read asynchronously and ordered by the
+// barrier waits and commits around the call, which are themselves volatile asm.
 QDEV void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                       uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 // Arrive once on `bar` when every MMA issued so far by this thread has completed.
 QDEV void mma_commit(uint64_t *bar) {

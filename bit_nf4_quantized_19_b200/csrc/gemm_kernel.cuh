@@ -15,9 +15,12 @@
 // accumulated to ~2^-16 relative precision, not bf16 precision.
 //
 // Warp roles (512 threads, one CTA per SM, persistent over tiles):
-//   warp 0        TMA producer: activation tiles (X / dY, or the LoRA hi/lo
-//                 operand) and packed 4-bit weight tiles + block constants.
+//   warp 0        TMA producer of the activation tiles (X / dY, or the LoRA
+//                 hi/lo operand).
 //   warp 1        TMEM allocator and single-thread MMA issuer.
+//   warp 2        TMA producer of the packed 4-bit weight tiles + block
+//                 constants (its own ring, so the small weight stream runs
+//                 ahead of the activation ring instead of waiting behind it).
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
 //   warps 8..15   dequant producers, two warpgroups taking alternate stages:
 //                 packed codes + block constant -> bf16 tile in the
@@ -34,9 +37,17 @@ constexpr int kGemmThreads = 512;
 constexpr int kBN = 256;                  // tokens per tile (MMA N)
 constexpr int kWT = 128;                  // weight-side rows per tile (MMA M)
 constexpr int kBK = 64;                   // contraction per stage (one quant block)
-constexpr int kStagesB = 4;               // activation ring
-constexpr int kStagesA = 4;               // dequantized weight ring
-constexpr int kStagesW = 4;               // packed code ring
+#ifndef QLORA_GEMM_STAGES
+#define QLORA_GEMM_STAGES 4
+#endif
+#ifndef QLORA_GEMM_STAGES_W
+#define QLORA_GEMM_STAGES_W 6
+#endif
+// The MMA stages: one ring of (activation tile, dequantized weight tile) pairs,
+// released by a single commit per stage.
+constexpr int kStagesB = QLORA_GEMM_STAGES;     // activation tiles (32 KB each)
+constexpr int kStagesA = QLORA_GEMM_STAGES;     // dequantized weight tiles (16 KB each)
+constexpr int kStagesW = QLORA_GEMM_STAGES_W;   // packed code + constant ring (4.5 KB stages)
 constexpr int kBStageBytes = kBN * 128;   // 32 KB
 constexpr int kAStageBytes = kWT * 128;   // 16 KB
 constexpr int kWStageBytes = 4096;        // packed codes of one stage
@@ -46,6 +57,8 @@ constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
 constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStagesB * kBStageBytes +
                                kStagesA * kAStageBytes + kStagesW * (kWStageBytes + kSStageBytes) +
                                1024 /*barriers, flags, levels*/;
+static_assert(kGemmSmemBytes <= 227 * 1024, "GEMM shared memory exceeds the per-CTA limit");
+static_assert(kStagesW <= 32 && kStagesB <= 32, "ring bookkeeping uses 32-bit masks");
 
 enum GemmMode : int { kModeFwd = 0, kModeDx = 1 };
 
@@ -79,10 +92,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t *sW = sA + kStagesA * kAStageBytes;
   float *sS = reinterpret_cast<float *>(sW + kStagesW * kWStageBytes);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sS + kStagesW * (kSStageBytes / 4));
-  uint64_t *full_B = bars;
-  uint64_t *empty_B = full_B + kStagesB;
-  uint64_t *full_A = empty_B + kStagesB;
-  uint64_t *empty_A = full_A + kStagesA;
+  uint64_t *full_B = bars;                  // activation tile landed (TMA)
+  uint64_t *full_A = full_B + kStagesB;     // dequantized tile written (4 warp arrivals)
+  uint64_t *empty_A = full_A + kStagesA;    // MMAs of the stage done: both tiles free
   uint64_t *full_W = empty_A + kStagesA;
   uint64_t *empty_W = full_W + kStagesW;
   uint64_t *tmem_full = empty_W + kStagesW;
@@ -97,10 +109,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = tid & 31;
 
   if (tid == 0) {
-    for (int i = 0; i < kStagesB; ++i) { mbar_init(&full_B[i], 1); mbar_init(&empty_B[i], 1); }
-    for (int i = 0; i < kStagesA; ++i) { mbar_init(&full_A[i], 128); mbar_init(&empty_A[i], 1); }
-    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 1); mbar_init(&empty_W[i], 128); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 128); }
+    for (int i = 0; i < kStagesA; ++i) {
+      mbar_init(&full_B[i], 1);
+      mbar_init(&full_A[i], 4);
+      mbar_init(&empty_A[i], 1);
+    }
+    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 1); mbar_init(&empty_W[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -126,18 +141,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = p.kb_main + p.kb_lora;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ activation producer
     if (lane == 0) {
-      int bs = 0, ws = 0;
-      uint32_t bph = 0, wph = 0;
-      uint32_t armedB = 0, armedW = 0;          // bit s: stage s armed at least once
-      uint32_t lastB = 0, lastW = 0;            // bit s: parity of the last arming
+      int bs = 0;
+      uint32_t bph = 0;
+      uint32_t armedB = 0, lastB = 0;          // bit s: armed at least once / parity of last arming
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int m0 = (tile / p.num_w_tiles) * kBN;
-        const int w0 = (tile % p.num_w_tiles) * kWT;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_bar(&empty_B[bs], bph ^ 1u, wt)) { ok = false; break; }
+          if (!wait_bar(&empty_A[bs], bph ^ 1u, wt)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_B[bs], kBStageBytes);
           if (kb < p.kb_main)
             tma_load_2d(sB + bs * kBStageBytes, &tm_act, &full_B[bs], kb * kBK, m0);
@@ -146,23 +159,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           armedB |= 1u << bs;
           lastB = (lastB & ~(1u << bs)) | (bph << bs);
           if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
-          if (kb < p.kb_main) {
-            if (!wait_bar(&empty_W[ws], wph ^ 1u, wt)) { ok = false; break; }
-            mbar_arrive_expect_tx(&full_W[ws], kWStageBytes + kSStageBytes);
-            if (MODE == kModeFwd) {
-              // codes: 32 bytes (64 values of K) x 128 weight rows; constants S[kb][w0 .. w0+128)
-              tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
-              tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], w0, kb);
-            } else {
-              // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..;
-              // constants S[w0/64 + {0,1}][kb*64 .. kb*64+64)
-              tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
-              tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], kb * kBK, w0 / kBK);
-            }
-            armedW |= 1u << ws;
-            lastW = (lastW & ~(1u << ws)) | (wph << ws);
-            if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
-          }
         }
       }
       // Every issued copy lands before the block may exit (bounded).
@@ -170,45 +166,84 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const Waiter final_wt{&no_abort, p.limit_ns};
       for (int s = 0; s < kStagesB; ++s)
         if (armedB & (1u << s)) wait_bar(&full_B[s], (lastB >> s) & 1u, final_wt);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ weight producer
+    if (lane == 0) {
+      int ws = 0;
+      uint32_t wph = 0;
+      uint32_t armedW = 0, lastW = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int w0 = (tile % p.num_w_tiles) * kWT;
+        for (int kb = 0; kb < p.kb_main; ++kb) {
+          if (!wait_bar(&empty_W[ws], wph ^ 1u, wt)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_W[ws], kWStageBytes + kSStageBytes);
+          if (MODE == kModeFwd) {
+            // codes: 32 bytes (64 values of K) x 128 weight rows; constants S[kb][w0 .. w0+128)
+            tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
+            tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], w0, kb);
+          } else {
+            // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..;
+            // constants S[w0/64 + {0,1}][kb*64 .. kb*64+64)
+            tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
+            tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], kb * kBK, w0 / kBK);
+          }
+          armedW |= 1u << ws;
+          lastW = (lastW & ~(1u << ws)) | (wph << ws);
+          if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
+        }
+      }
+      volatile int no_abort = 0;
+      const Waiter final_wt{&no_abort, p.limit_ns};
       for (int s = 0; s < kStagesW; ++s)
         if (armedW & (1u << s)) wait_bar(&full_W[s], (lastW >> s) & 1u, final_wt);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // A lean loop: descriptors of stage 0 are built once; a stage adds its byte
+    // offset >> 4 to the start-address field, a K=16 step adds 32 B (K-major)
+    // or 4096 B (MN-major, two 8-row groups) >> 4; one commit per stage frees
+    // both tiles of the stage.
     if (lane == 0) {
       constexpr uint32_t idesc_main = make_idesc_bf16(kWT, kBN, MODE == kModeDx, false);
       constexpr uint32_t idesc_lora = make_idesc_bf16(kWT, kBN, MODE == kModeFwd, false);
-      int as = 0, bs = 0, acc = 0;
-      uint32_t aph = 0, bph = 0, accph = 0;
-      bool ok = true;
+      constexpr uint32_t a_step_main = (MODE == kModeDx) ? (4096u >> 4) : (32u >> 4);
+      constexpr uint32_t a_step_lora = (MODE == kModeFwd) ? (4096u >> 4) : (32u >> 4);
+      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+      const uint64_t ad_main0 = (MODE == kModeDx) ? sw128_desc(a0, 1024, 2048) : sw128_desc(a0, 16, 1024);
+      const uint64_t ad_lora0 = (MODE == kModeFwd) ? sw128_desc(a0, 1024, 2048) : sw128_desc(a0, 16, 1024);
+      const uint64_t bd0 = sw128_desc(b0, 16, 1024);
+      const int kb_main = p.kb_main, kb_lora = p.kb_lora;
       const int lora_steps_total = (2 * p.r) / 16;
+      int st = 0, acc = 0;
+      uint32_t ph = 0, accph = 0;
+      bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         if (!wait_bar(&tmem_empty[acc], accph ^ 1u, wt)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_bar(&full_A[as], aph, wt) || !wait_bar(&full_B[bs], bph, wt)) { ok = false; break; }
+        for (int kb = 0; kb < kb_main; ++kb) {
+          if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + as * kAStageBytes);
-          const uint32_t b_base = smem_u32(sB + bs * kBStageBytes);
-          const bool main = kb < p.kb_main;
-          int nk = 4;
-          if (!main) {
-            const int done = (kb - p.kb_main) * 4;
-            nk = min(4, lora_steps_total - done);
-          }
-          for (int k = 0; k < nk; ++k) {
-            const bool a_mn = main ? (MODE == kModeDx) : (MODE == kModeFwd);
-            const uint64_t adesc = a_mn ? sw128_desc(a_base + k * 4096, 1024, 2048)
-                                        : sw128_desc(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = sw128_desc(b_base + k * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, adesc, bdesc, main ? idesc_main : idesc_lora,
-                        (kb > 0 || k > 0) ? 1u : 0u);
-          }
-          mma_commit(&empty_A[as]);
-          mma_commit(&empty_B[bs]);
-          if (++as == kStagesA) { as = 0; aph ^= 1u; }
-          if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
+          const uint64_t ad = ad_main0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
+          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStageBytes >> 4));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(d_tmem, ad + k * a_step_main, bd + k * 2, idesc_main, (kb | k) ? 1u : 0u);
+          mma_commit(&empty_A[st]);
+          if (++st == kStagesA) { st = 0; ph ^= 1u; }
+        }
+        for (int ls = 0; ok && ls < kb_lora; ++ls) {
+          if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = ad_lora0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
+          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStageBytes >> 4));
+          const int nk = min(4, lora_steps_total - ls * 4);
+          for (int k = 0; k < nk; ++k)
+            mma_bf16_ss(d_tmem, ad + k * a_step_lora, bd + k * 2, idesc_lora, 1u);
+          mma_commit(&empty_A[st]);
+          if (++st == kStagesA) { st = 0; ph ^= 1u; }
         }
         if (!ok) break;
         mma_commit(&tmem_full[acc]);
@@ -251,7 +286,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tmem_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tmem_empty[acc]);
       if (++acc == 2) { acc = 0; accph ^= 1u; }
     }
   } else if (warp >= 8) {
@@ -275,7 +311,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (main) {
           const int ws = static_cast<int>(my_w % kStagesW);
           const uint32_t wph = (my_w / kStagesW) & 1u;
-          if (!wait_bar(&full_W[ws], wph, wt) || !wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+          // warp-uniform: the per-warp arrivals below need every lane on the same path
+          const bool w_ok = wait_bar(&full_W[ws], wph, wt) && wait_bar(&empty_A[as], aph ^ 1u, wt);
+          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
           uint32_t src, dst;
           int swz;
           float sc;
@@ -296,7 +334,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint4 c0 = ld_shared_v4(src);
           const uint4 c1 = ld_shared_v4(src + 16);
-          mbar_arrive(&empty_W[ws]);        // codes are in registers now
+          __syncwarp();                     // the warp's codes are in registers now
+          if (lane == 0) mbar_arrive(&empty_W[ws]);
           Nf4Lut lut;
           nf4_build_lut(L, sc, lut);
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -307,11 +346,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             st_shared_v4(dst + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
           }
           fence_proxy_async_smem();
-          mbar_arrive(&full_A[as]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_A[as]);
         } else {
           // LoRA weight-side stage: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
           const int ls = kb - p.kb_main;
-          if (!wait_bar(&empty_A[as], aph ^ 1u, wt)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, wait_bar(&empty_A[as], aph ^ 1u, wt))) { ok = false; break; }
           const uint32_t abase = smem_u32(sA + as * kAStageBytes);
           if (MODE == kModeFwd) {
             // MN-major: K index cr (0..63), M group mg: B[c mod r][w0 + 64 mg ..]
@@ -338,7 +378,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          mbar_arrive(&full_A[as]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_A[as]);
         }
       }
     }

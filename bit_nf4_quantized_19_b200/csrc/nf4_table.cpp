@@ -62,7 +62,8 @@ Nf4Tables build() {
     const double mid = 0.5 * (static_cast<double>(T.levels[i]) + static_cast<double>(T.levels[i + 1]));
     T.thresholds[i] = round_down_f32(mid);
   }
-  // Bin table for the quantizer: bin j covers 32*xn in [j-32.5, j-31.5].
+  // Bin table for the quantizer: bin j (stored at (j - 32) mod 128) covers
+  // 32*xn in [j-32.5, j-31.5].
   for (int j = 0; j < kQuantBins; ++j) {
     T.bins[j].t = 2.0f;
     T.bins[j].c = 0;
@@ -81,8 +82,13 @@ Nf4Tables build() {
       }
     }
     if (inside > 1) ok = false;
-    T.bins[j].t = tin;
-    T.bins[j].c = below;
+    const int slot = (j - 32) & (kQuantBins - 1);
+    T.bins[slot].t = tin;
+    T.bins[slot].c = below;
+  }
+  for (int k = 0; k < 128; ++k) {
+    volatile float m = 1.0f + static_cast<float>(k) / 128.0f;
+    T.rcp[k] = 1.0f / m;  // IEEE single division: RN32(1/m)
   }
   T.ok = ok;
   return T;

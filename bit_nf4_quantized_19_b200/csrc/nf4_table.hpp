@@ -5,10 +5,10 @@
 namespace qlora {
 
 // One entry of the quantizer's bin table.  The normalised value xn in [-1, 1]
-// falls in bin j = round_half_even(32 * xn) + 32 (0..64).  Each bin holds at
-// most one decision threshold, so the code is  c + (xn > t)  with t = +2 for a
-// bin without a threshold.  Entries 65..127 exist only so that a masked index
-// computed from a non-finite value stays inside the table.
+// falls in bin j = round_half_even(32 * xn) (-32..32), stored at index j mod 128.
+// Each bin holds at most one decision threshold, so the code is  c + (xn > t)
+// with t = +2 for a bin without a threshold.  The unused indices exist only so
+// that a masked index computed from a non-finite value stays inside the table.
 struct QuantBin {
   float t;
   int32_t c;
@@ -19,6 +19,7 @@ struct Nf4Tables {
   float levels[16];      // ascending, levels[0] = -1, levels[7] = 0, levels[15] = 1
   float thresholds[15];  // RD32((levels[i] + levels[i+1]) / 2)
   QuantBin bins[kQuantBins];
+  float rcp[128];        // RN32(1 / (1 + k/128)), k = 0..127
   bool ok;               // construction invariants held
 };
 

@@ -437,6 +437,7 @@ qlora_status qlora_nf4_quantize(const uint16_t *W, int64_t rows, int64_t cols,
   if (!T.ok) return QLORA_ERR_DEVICE_CHECK;
   QuantTables tab;
   std::memcpy(tab.bins, T.bins, sizeof(tab.bins));
+  std::memcpy(tab.rcp, T.rcp, sizeof(tab.rcp));
   const int64_t n = rows * cols;
   const int64_t groups = (n + kGroupElems - 1) / kGroupElems;
   if (groups > 0x7FFFFFFFll) return QLORA_ERR_UNSUPPORTED_SHAPE;

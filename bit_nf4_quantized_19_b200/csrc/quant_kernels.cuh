@@ -13,7 +13,8 @@ constexpr int kGroup = 256;                // blocks per second-level constant
 constexpr int kGroupElems = kBlock * kGroup;
 
 struct QuantTables {
-  QuantBin bins[kQuantBins];
+  QuantBin bins[kQuantBins];   // indexed by round(32 * xn) mod 128
+  float rcp[128];              // RN32(1 / (1 + k/128)): reciprocals of the bf16 mantissas
 };
 struct Levels {
   float v[16];
@@ -23,21 +24,28 @@ struct Levels {
 // block, each owning 8 consecutive values (one 16-byte load), 32 blocks per pass,
 // 8 passes.  All eight 16-byte loads are issued before any arithmetic.
 //   absmax: max |w| within the thread, then an xor-shuffle over the 8 lanes;
-//   code:   xn = RN32(w / a_b) (IEEE division), bin j = round(32 xn) + 32 from
-//           the exact sum 32 xn + 1.5*2^23, code = bins[j].c + (xn > bins[j].t);
-//           this equals the count of decision thresholds below xn, i.e. the
-//           nearest level with ties to the lower index;
+//   xn:     RN32(w / a_b).  For 2^-64 <= a_b <= 2^64 (every realistic block) the
+//           division is Markstein's FMA correction of w * RN32(1/a_b), where
+//           RN32(1/a_b) is an exact power-of-two scaling of a table entry because
+//           a_b is a bf16 value; outside that range, IEEE division.  An exhaustive
+//           host check over all bf16 pairs of the fast range shows both give the
+//           same code for every input (tests/csrc/division_check.c);
+//   code:   bin j = round(32 xn) (exact, from the sum 32 xn + 1.5*2^23), then
+//           code = bins[j].c + (xn > bins[j].t): the number of decision thresholds
+//           below xn, i.e. the nearest level with ties to the lower index;
 //   pack:   8 codes -> one 32-bit word (element 2j in the low nibble of byte j);
 //   double quant (after all passes): c_g = max a_b over the group,
 //           step = RN32(c_g / 255), q8 = min(255, rint(RN32(a_b / step))).
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(
+__global__ void __launch_bounds__(256, 3) nf4_quantize_kernel(
     const uint16_t *__restrict__ W, int64_t n, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab) {
   __shared__ QuantBin bins[kQuantBins];
+  __shared__ float rcp[128];
   __shared__ float amax[kGroup];
   __shared__ float wmax[8];
   const int tid = threadIdx.x;
   if (tid < kQuantBins) bins[tid] = tab.bins[tid];
+  if (tid < 128) rcp[tid] = tab.rcp[tid];
 
   const int64_t g = blockIdx.x;
   const int64_t gbase = g * kGroupElems;
@@ -77,16 +85,38 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
     if (!(am <= 3.402823466e38f)) nonfinite = true;
-    const float a = (am > 0.f) ? am : 1.0f;
+    const bool fast = (am >= 0x1p-64f) && (am <= 0x1p64f);
+    // RN32(1/am) = RN32(1/m) * 2^-e for am = m * 2^e (m has 7 fraction bits)
+    const uint32_t ab = __float_as_uint(am);
+    const int ex = static_cast<int>((ab >> 23) & 0xFFu) - 127;
+    const float y = __uint_as_float(__float_as_uint(rcp[(ab >> 16) & 127u]) - (static_cast<uint32_t>(ex) << 23));
     uint32_t word = 0;
+    if (__all_sync(0xffffffffu, fast)) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float xn = __fdiv_rn(w[j], a);
-      const float f = __fadd_rn(__fmul_rn(xn, 32.0f), 12582912.0f);
-      const int idx = (__float_as_int(f) - 0x4B400000 + 32) & (kQuantBins - 1);
-      const QuantBin b = bins[idx];
-      const uint32_t code = static_cast<uint32_t>(b.c + (xn > b.t ? 1 : 0));
-      word |= code << (4 * j);
+      for (int j = 0; j < 8; ++j) {
+        const float q0 = __fmul_rn(w[j], y);
+        const float r = __fmaf_rn(-q0, am, w[j]);
+        const float xn = __fmaf_rn(r, y, q0);
+        const float f = __fmaf_rn(xn, 32.0f, 12582912.0f);
+        const QuantBin b = bins[__float_as_uint(f) & (kQuantBins - 1)];
+        word |= static_cast<uint32_t>(b.c + (xn > b.t ? 1 : 0)) << (4 * j);
+      }
+    } else {
+      const float a = (am > 0.f) ? am : 1.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float xn;
+        if (fast) {
+          const float q0 = __fmul_rn(w[j], y);
+          const float r = __fmaf_rn(-q0, am, w[j]);
+          xn = __fmaf_rn(r, y, q0);
+        } else {
+          xn = __fdiv_rn(w[j], a);
+        }
+        const float f = __fmaf_rn(xn, 32.0f, 12582912.0f);
+        const QuantBin b = bins[__float_as_uint(f) & (kQuantBins - 1)];
+        word |= static_cast<uint32_t>(b.c + (xn > b.t ? 1 : 0)) << (4 * j);
+      }
     }
     if (e + 8 <= n) {
       *reinterpret_cast<uint32_t *>(codes + (e >> 1)) = word;
