@@ -36,6 +36,7 @@ WORKLOAD = ("LLaMA-7B-shaped projections W[N,K] in {4096x4096, 11008x4096, 4096x
 FLUSH_BYTES = 256 << 20
 SKINNY = [(m, n, 4096) for n in (4096, 11008) for m in (1, 4, 16)]
 BIG_N = 1_000_000_000
+GRAPH_STREAM_BYTES = 320 << 20   # weights streamed per graph replay of the decode measurement
 
 
 def step_flops(M, N, K, r):
@@ -461,7 +462,7 @@ def hbm_subpaths(q, torch, dev, stream, P, flush):
         XA = torch.empty(M, r, dtype=torch.float32, device=dev)
         ws = q.make_workspace(M, N, K, r, dev)
         for _ in range(3):
-            q.linear_fwd(X, Wq, A, B, r and 2.0, workspace=ws, Y=Y, XA=XA)
+            q.linear_fwd(X, Wq, A, B, 2.0, workspace=ws, Y=Y, XA=XA)
         ts = []
         for i in range(20):
             flush.fill_(float(i))
@@ -476,6 +477,48 @@ def hbm_subpaths(q, torch, dev, stream, P, flush):
         out[f"skinny_M{M}_{N}x{K}"] = {"ms": t, "GB/s": by / t / 1e6, "frac": by / t / 1e6 / P["hbm"],
                                        "bytes": by}
         del Wb, Wq
+    # skinny forward inside one CUDA graph: L distinct weights whose NF4 storage
+    # together exceeds 2.5x the L2, called back to back as the consecutive layers of
+    # a decode step are, so every call streams its weight from HBM
+    for (N, K) in sorted({(n, k) for _, n, k in SKINNY}):
+        r = RANK_R
+        Wb = (torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        Wq0 = q.nf4_quantize(Wb)
+        L = max(8, -(-GRAPH_STREAM_BYTES // Wq0.nbytes))
+        Wqs = [Wq0] + [q.nf4_quantize(Wb) for _ in range(L - 1)]
+        del Wb
+        for M in sorted({m for m, n, k in SKINNY if (n, k) == (N, K)}):
+            X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
+            A = (torch.randn(K, r, generator=gen, device=dev) / r).to(torch.bfloat16)
+            B = (torch.randn(r, N, generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            XA = torch.empty(M, r, dtype=torch.float32, device=dev)
+            ws = q.make_workspace(M, N, K, r, dev)
+            for Wq in Wqs:
+                q.linear_fwd(X, Wq, A, B, 2.0, workspace=ws, Y=Y, XA=XA)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for Wq in Wqs:
+                    q.linear_fwd(X, Wq, A, B, 2.0, workspace=ws, Y=Y, XA=XA)
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            reps = 10
+            cur = torch.cuda.current_stream()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(cur)
+            for _ in range(reps):
+                graph.replay()
+            b.record(cur)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b) / (reps * L)
+            by = Wqs[0].nbytes + 2 * M * K + 2 * M * N + 2 * K * r + 2 * r * N + 4 * M * r
+            out[f"skinny_graph_M{M}_{N}x{K}"] = {"ms": t, "GB/s": by / t / 1e6, "frac": by / t / 1e6 / P["hbm"],
+                                                 "bytes": by, "layers": L}
+            del graph
+        del Wqs, Wq0
+        torch.cuda.empty_cache()
     out["hbm_peak_GBps"] = P["hbm"]
     out["hbm_peak_source"] = P["src"]
     return out

@@ -11,17 +11,33 @@
 #include "lora_mma.cuh"
 #include "nf4_table.hpp"
 #include "quant_kernels.cuh"
+#include "skinny_kernel.cuh"
 
 using namespace qlora;
 
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+constexpr int64_t kSkinnyMaxTokens = 16;   // forward with at most this many tokens: one-launch kernel
 std::atomic<uint32_t> g_wait_limit_us{2000000u};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+#ifndef QLORA_SKINNY_CLUSTER
+#define QLORA_SKINNY_CLUSTER 8
+#endif
+constexpr int kSkSmemLimit = 200 * 1024;
+
+template <int C>
+cudaError_t set_skinny_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(qlora_skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSkSmemLimit);
+  if (e == cudaSuccess && C > 8)
+    e = cudaFuncSetAttribute(qlora_skinny_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
 
 struct DeviceInfo {
   int sms = 0;
@@ -52,6 +68,10 @@ qlora_status device_info(DeviceInfo **out) {
                              kGemmSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    if (set_skinny_attrs<1>() != cudaSuccess || set_skinny_attrs<2>() != cudaSuccess ||
+        set_skinny_attrs<4>() != cudaSuccess || set_skinny_attrs<8>() != cudaSuccess ||
+        set_skinny_attrs<16>() != cudaSuccess)
       return QLORA_ERR_CUDA;
     d.gemm_attr_set = true;
   }
@@ -328,6 +348,103 @@ qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT,
   return cuda_status(cudaGetLastError());
 }
 
+// Few-token forward: one cluster launch, no workspace.  Clusters of C CTAs
+// (power of two, 8 preferred, 16 when the slice would not fit) split K into C
+// slices of ks (a multiple of 256) values.  False when no plan fits: the caller
+// then takes the general path.
+bool skinny_choose(int64_t M, int64_t K, int r, SkinnyPlan &pl) {
+  const int64_t macro = (K + kSkMacro - 1) / kSkMacro;
+  int C = QLORA_SKINNY_CLUSTER;
+  while (C > 1 && C > macro) C >>= 1;
+  for (; C <= kSkMaxCluster; C <<= 1)
+    if (skinny_plan_for(static_cast<int>(M), static_cast<int>(K), r, C, kSkSmemLimit, pl)) return true;
+  return false;
+}
+
+// 16-CTA clusters are not portable: take one only where the device can place it.
+bool skinny_launchable(const SkinnyPlan &pl, int64_t N) {
+  if (pl.C <= 8) return true;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.C), static_cast<unsigned>(N / kSkRows), 1);
+  cfg.blockDim = dim3(kSkThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(pl.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, qlora_skinny_kernel<16>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return n > 0;
+}
+
+qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, const uint16_t *A,
+                           const uint16_t *B, int r, float s, uint16_t *Y, float *XA_out,
+                           const SkinnyPlan &pl, cudaStream_t st) {
+  const int64_t N = Wq->rows, K = Wq->cols;
+  SkinnyParams p{};
+  p.X = X;
+  p.codes = Wq->codes;
+  p.q8 = Wq->q8;
+  p.step = Wq->step;
+  p.A = A;
+  p.B = B;
+  p.Y = Y;
+  p.XA_out = XA_out;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(K);
+  p.N = static_cast<int>(N);
+  p.r = r;
+  p.ks = pl.ks;
+  p.ka = pl.ka;
+  p.abox = pl.abox;
+  p.xpitch = pl.xpitch;
+  p.off_x = pl.off_x;
+  p.off_a = pl.off_a;
+  p.off_b = pl.off_b;
+  p.off_part = pl.off_part;
+  p.off_xa = pl.off_xa;
+  p.off_slot = pl.off_slot;
+  p.off_bar = pl.off_bar;
+  p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
+  p.s = s;
+  std::memcpy(p.levels, nf4_tables().levels, sizeof(p.levels));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.C), static_cast<unsigned>(N / kSkRows), 1);
+  cfg.blockDim = dim3(kSkThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(pl.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LaunchTimer lt(QLORA_K_SKINNY, st);
+  const int R = kSkRows / pl.C;
+  CUtensorMap tm_codes, tm_a, tm_b;
+  if (!make_map_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, kSkMacro / 2,
+                   kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, 2 * r, r, pl.abox,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, 2 * N, R, r, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QLORA_ERR_CUDA;
+  switch (pl.C) {
+    case 1: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<1>, tm_codes, tm_a, tm_b, p));
+    case 2: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<2>, tm_codes, tm_a, tm_b, p));
+    case 4: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<4>, tm_codes, tm_a, tm_b, p));
+    case 8: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<8>, tm_codes, tm_a, tm_b, p));
+    case 16: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<16>, tm_codes, tm_a, tm_b, p));
+    default: return QLORA_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
 // One fused GEMM launch.  MODE fwd: Y = X deq(W)^T + LoRA; MODE dx: dX = dY deq(W) + LoRA.
 template <int MODE>
 qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, const float *S,
@@ -492,6 +609,10 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t N = Wq->rows, K = Wq->cols;
   if (!workspace || workspace_bytes < fwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
+  if (M <= kSkinnyMaxTokens) {
+    SkinnyPlan pl{};
+    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) return launch_skinny(X, M, Wq, A, B, r, s, Y, XA_out, pl, stream);
+  }
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
