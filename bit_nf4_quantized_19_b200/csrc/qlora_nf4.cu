@@ -69,7 +69,10 @@ qlora_status device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if (set_skinny_attrs<1>() != cudaSuccess || set_skinny_attrs<2>() != cudaSuccess ||
+    if (cudaFuncSetAttribute(qlora_xa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             xa_smem_bytes(64) > xa_smem_bytes(128) ? xa_smem_bytes(64) : xa_smem_bytes(128)) !=
+            cudaSuccess ||
+        set_skinny_attrs<1>() != cudaSuccess || set_skinny_attrs<2>() != cudaSuccess ||
         set_skinny_attrs<4>() != cudaSuccess || set_skinny_attrs<8>() != cudaSuccess ||
         set_skinny_attrs<16>() != cudaSuccess)
       return QLORA_ERR_CUDA;
@@ -384,32 +387,56 @@ bool skinny_launchable(const SkinnyPlan &pl, int64_t N) {
 }
 
 qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, const uint16_t *A,
-                           const uint16_t *B, int r, float s, uint16_t *Y, float *XA_out,
+                           const uint16_t *B, int r, float s, uint16_t *Y, float *xa,
                            const SkinnyPlan &pl, cudaStream_t st) {
   const int64_t N = Wq->rows, K = Wq->cols;
+  // 1. XA = X A by one cluster; it lets the dependent launch below start at once
+  {
+    XaParams xp{};
+    xp.X = X;
+    xp.A = A;
+    xp.xa = xa;
+    xp.M = static_cast<int>(M);
+    xp.K = static_cast<int>(K);
+    xp.r = r;
+    xp.kx = static_cast<int>((K / kXaCluster + 15) / 16 * 16);
+    xp.chunk = xa_chunk_rows(r);
+    xp.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(kXaCluster, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(xa_smem_bytes(r));
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kXaCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchTimer lt(QLORA_K_PROJECT, st);
+    const qlora_status e = cuda_status(cudaLaunchKernelEx(&cfg, qlora_xa_kernel, xp));
+    if (e != QLORA_OK) return e;
+  }
+  // 2. the weight pass, a programmatic dependent of the XA launch
   SkinnyParams p{};
   p.X = X;
   p.codes = Wq->codes;
   p.q8 = Wq->q8;
   p.step = Wq->step;
-  p.A = A;
   p.B = B;
+  p.xa = xa;
   p.Y = Y;
-  p.XA_out = XA_out;
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.N = static_cast<int>(N);
   p.r = r;
   p.ks = pl.ks;
-  p.ka = pl.ka;
-  p.abox = pl.abox;
   p.xpitch = pl.xpitch;
-  p.off_x = pl.off_x;
-  p.off_a = pl.off_a;
   p.off_b = pl.off_b;
+  p.off_x = pl.off_x;
   p.off_part = pl.off_part;
   p.off_xa = pl.off_xa;
-  p.off_slot = pl.off_slot;
   p.off_bar = pl.off_bar;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
   p.s = s;
@@ -419,28 +446,28 @@ qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, 
   cfg.blockDim = dim3(kSkThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(pl.C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   LaunchTimer lt(QLORA_K_SKINNY, st);
   const int R = kSkRows / pl.C;
-  CUtensorMap tm_codes, tm_a, tm_b;
+  CUtensorMap tm_codes, tm_b;
   if (!make_map_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, kSkMacro / 2,
                    kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, 2 * r, r, pl.abox,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, 2 * N, R, r, CU_TENSOR_MAP_SWIZZLE_NONE))
     return QLORA_ERR_CUDA;
   switch (pl.C) {
-    case 1: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<1>, tm_codes, tm_a, tm_b, p));
-    case 2: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<2>, tm_codes, tm_a, tm_b, p));
-    case 4: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<4>, tm_codes, tm_a, tm_b, p));
-    case 8: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<8>, tm_codes, tm_a, tm_b, p));
-    case 16: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<16>, tm_codes, tm_a, tm_b, p));
+    case 1: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<1>, tm_codes, tm_b, p));
+    case 2: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<2>, tm_codes, tm_b, p));
+    case 4: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<4>, tm_codes, tm_b, p));
+    case 8: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<8>, tm_codes, tm_b, p));
+    case 16: return cuda_status(cudaLaunchKernelEx(&cfg, qlora_skinny_kernel<16>, tm_codes, tm_b, p));
     default: return QLORA_ERR_UNSUPPORTED_SHAPE;
   }
 }
@@ -611,7 +638,12 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
   if (!workspace || workspace_bytes < fwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
   if (M <= kSkinnyMaxTokens) {
     SkinnyPlan pl{};
-    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) return launch_skinny(X, M, Wq, A, B, r, s, Y, XA_out, pl, stream);
+    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) {
+      Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
+      float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
+      if (!xa) return QLORA_ERR_WORKSPACE;
+      return launch_skinny(X, M, Wq, A, B, r, s, Y, xa, pl, stream);
+    }
   }
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));

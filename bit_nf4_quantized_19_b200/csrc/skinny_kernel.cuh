@@ -1,29 +1,35 @@
-// Few-token forward (M <= 16 tokens) of the QLoRA linear layer, one launch:
+// Few-token forward (M <= 16 tokens) of the QLoRA linear layer:
 //     Y = X deq(W)^T + s (X A) B       ("QLoRA", ozercemkelahmet.com, How it works, Step 5)
 // The work is bound by reading the packed 4-bit weight from HBM (0.52 bytes per
 // weight) and by the instructions that decode it, so the design keeps every
-// other cost off that path:
-//   * each CTA owns 128 weight rows and one slice of K; the C CTAs of one weight
-//     tile form a thread-block cluster along K and reduce their fp32 partial
-//     results through distributed shared memory, in rank order (deterministic,
-//     no global scratch, no second launch);
-//   * the code slice arrives by TMA, one 128-row x 128-byte box (128B swizzle)
-//     per 256-value macro-block, each on its own mbarrier, so a warp starts on
-//     macro-block mb as soon as that box has landed; A and this rank's columns of
-//     B arrive by TMA as well; the block constants are prefetched by each lane
-//     into registers a few macro-blocks ahead; only the M real token rows of X
-//     are staged (the fragments of absent tokens are zero registers);
-//   * the NF4 codes are decoded in registers straight into the A-fragment layout
-//     of mma.sync m16n8k16 (weight rows on M, tokens on N).  The contraction
-//     index is permuted inside each macro-block so that the four lanes sharing a
-//     fragment row each hold one whole 64-value block: lane c of a row group
-//     takes block 4*mb + c, elements 4s..4s+3 at k-step s.  The 16-entry table
-//     bf16_RN(RN32(L[c] * RN32(q8 * step))) (the per-element definition of the
-//     dequantized weight) is then built once per 64 decoded values instead of
-//     once per 16.  X is read with the same permutation, so the sum is the plain
-//     dot product over K taken in another order;
-//   * XA = X A for the slice is a second small tensor-core product; the LoRA term
-//     s * XA B is added in fp32 during the cluster reduction.
+// other cost off that path.  Two launches:
+//   * qlora_xa_kernel: XA = X A (fp32 [M, r]) by one cluster of 8 CTAs, K split
+//     across the cluster and reduced through distributed shared memory in rank
+//     order.  It lets its dependent launch start at once;
+//   * qlora_skinny_kernel, launched as that dependent (programmatic dependent
+//     launch): everything it reads before its grid-dependency wait was written
+//     by kernels that finished before the XA kernel started, and it reads XA only
+//     after the wait, so the rank-r product runs beside it at no cost to it:
+//     - each CTA owns 128 weight rows and one slice of K; the C CTAs of one
+//       weight tile form a thread-block cluster along K and push their fp32
+//       partial results into the shared memory of the rank that finishes those
+//       rows, which sums them in rank order (deterministic, no global scratch);
+//     - the code slice arrives by TMA, one 128-row x 128-byte box (128B
+//       swizzle) per 256-value macro-block, each on its own mbarrier, so a warp
+//       starts on macro-block mb as soon as that box has landed; this rank's
+//       columns of B arrive by TMA too; the block constants are prefetched by
+//       each lane into registers a few macro-blocks ahead; only the M real token
+//       rows of X are staged (the fragments of absent tokens are zero registers);
+//     - the NF4 codes are decoded in registers straight into the A-fragment
+//       layout of mma.sync m16n8k16 (weight rows on M, tokens on N).  The
+//       contraction index is permuted inside each macro-block so that the four
+//       lanes sharing a fragment row each hold one whole 64-value block: lane c
+//       of a row group takes block 4*mb + c, elements 4s..4s+3 at k-step s.  The
+//       16-entry table bf16_RN(RN32(L[c] * RN32(q8 * step))) (the per-element
+//       definition of the dequantized weight) is then built once per 64 decoded
+//       values instead of once per 16.  X is read with the same permutation, so
+//       the sum is the plain dot product over K taken in another order;
+//     - the LoRA term s * XA B is added in fp32 when the owner finishes a row.
 #pragma once
 #include "common.cuh"
 
@@ -41,16 +47,13 @@ struct SkinnyParams {
   const uint8_t *codes;   // packed NF4 of W [N, K]
   const uint8_t *q8;
   const float *step;
-  const uint16_t *A;      // [K, r] bf16
   const uint16_t *B;      // [r, N] bf16
+  const float *xa;        // [M, r] fp32, written by qlora_xa_kernel
   uint16_t *Y;            // [M, N] bf16
-  float *XA_out;          // [M, r] fp32 or null
   int M, K, N, r;
   int ks;                 // K per cluster rank, a multiple of 256
-  int ka;                 // rows of A staged per pass, a multiple of abox
-  int abox;               // rows of A per TMA box (<= 256)
   int xpitch;             // X row pitch, bf16 elements; element k sits at k + 4 (k / 64)
-  int off_x, off_a, off_b, off_part, off_xa, off_slot, off_bar;  // byte offsets from the 1024-aligned base
+  int off_b, off_x, off_part, off_xa, off_bar;   // byte offsets from the 1024-aligned base
   uint64_t limit_ns;      // limit of every mbarrier wait
   float s;
   float levels[16];
@@ -103,8 +106,8 @@ QDEV int sk_xoff(int k) { return k + 4 * (k >> 6); }
 
 template <int C>
 __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
-    const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_a,
-    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ SkinnyParams p) {
+    const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_b,
+    const __grid_constant__ SkinnyParams p) {
   extern __shared__ __align__(16) uint8_t sk_raw[];
   uint8_t *sm = sk_raw + ((1024u - (smem_u32(sk_raw) & 1023u)) & 1023u);   // SW128 boxes need 1024 B
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -119,20 +122,22 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
   const int xp = p.xpitch;
   constexpr int R = kSkRows / C;                             // output rows finished by each rank
 
-  uint16_t *sX = reinterpret_cast<uint16_t *>(sm + p.off_x);       // [M][xp]
-  uint8_t *sA = sm + p.off_a;
   uint16_t *sB = reinterpret_cast<uint16_t *>(sm + p.off_b);       // [r][R]
+  uint16_t *sX = reinterpret_cast<uint16_t *>(sm + p.off_x);       // [M][xp]
   float *sRecv = reinterpret_cast<float *>(sm + p.off_part);       // [C ranks][R rows][16 tokens]
-  float *sXA = reinterpret_cast<float *>(sm + p.off_xa);           // [16][r] partial, then [16][r] sum
-  float *sSlot = reinterpret_cast<float *>(sm + p.off_slot);       // [8 warps][16][8]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + p.off_bar);   // [nmb] codes, then one for A/B
-  uint64_t *bar_ab = bars + (p.ks / kSkMacro);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_ab + 1);
+  float *sXA = reinterpret_cast<float *>(sm + p.off_xa);           // [M][r]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + p.off_bar);   // [nmb] codes, then one for B
+  uint64_t *bar_b = bars + (p.ks / kSkMacro);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_b + 1);
   const Waiter waiter{abort_flag, p.limit_ns};
 
   // ---- 1. every load of the CTA is issued first: X by all threads (cp.async,
   //         8 bytes each: an 8-byte piece never straddles a 64-value block of the
-  //         padded layout), the bulk copies by one thread, A and B before the codes
+  //         padded layout); by one thread the code boxes, then this rank's B columns
+  if (tid == 32) {
+    prefetch_tmap(&tm_codes);
+    prefetch_tmap(&tm_b);
+  }
   for (int t = warp; t < p.M; t += kSkThreads / 32) {
     const uint16_t *xr = p.X + static_cast<int64_t>(t) * p.K + k0;
     const uint32_t xs = smem_u32(sX + t * xp);
@@ -142,21 +147,15 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
   if (tid == 0) {
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_codes);
     *abort_flag = 0;
     for (int i = 0; i <= p.ks / kSkMacro; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    const int a_first = min(kn, p.ka);
-    const uint32_t a_bytes = static_cast<uint32_t>((a_first + p.abox - 1) / p.abox * p.abox * p.r * 2);
-    mbar_arrive_expect_tx(bar_ab, a_bytes + static_cast<uint32_t>(p.r * R * 2));
-    for (int a = 0; a < a_first; a += p.abox) tma_load_2d(sA + a * p.r * 2, &tm_a, bar_ab, 0, k0 + a);
-    tma_load_2d(sB, &tm_b, bar_ab, w0 + static_cast<int>(rank) * R, 0);
     for (int mb = 0; mb < nmb; ++mb) {
       mbar_arrive_expect_tx(&bars[mb], kSkBoxBytes);
       tma_load_2d(sm + mb * kSkBoxBytes, &tm_codes, &bars[mb], (k0 >> 1) + mb * (kSkMacro / 2), w0);
     }
+    mbar_arrive_expect_tx(bar_b, static_cast<uint32_t>(p.r * R * 2));
+    tma_load_2d(sB, &tm_b, bar_b, w0 + static_cast<int>(rank) * R, 0);
   }
   // block constants of this lane's rows, kSkPre macro-blocks ahead (raw q8 and step)
   const int ra = warp * 16 + g, rb = ra + 8;
@@ -182,76 +181,13 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();   // barrier init and X visible to every warp
 
-  // ---- 2. XA partial over this K slice while the codes are in flight: tokens on
-  // M (16), adapter columns on N in jt tiles of 8; with fewer than 8 tiles the K
-  // steps of a tile are split over nsplit warps and summed in warp order later.
+  // ---- 2. main product over the macro-blocks
   const bool tok0 = g < p.M, tok1 = g + 8 < p.M;
-  const int jt = p.r >> 3;
-  const int nsplit = jt >= 8 ? 1 : 8 / jt;
-  const int my_t8 = (jt >= 8) ? warp : warp / nsplit, my_part = (jt >= 8) ? 0 : warp % nsplit;
-  const bool xa_active = (jt >= 8) || (warp < jt * nsplit);
-  float xacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  bool ok = true;
-  for (int pass = 0, a0 = 0; pass == 0 || a0 < kn; ++pass, a0 += p.ka) {
-    const int arows = max(0, min(p.ka, kn - a0));
-    if (pass > 0) {                                // later passes of A (only when the slice exceeds ka)
-      __syncthreads();
-      if (tid == 0) {
-        mbar_arrive_expect_tx(bar_ab, static_cast<uint32_t>((arows + p.abox - 1) / p.abox * p.abox * p.r * 2));
-        for (int a = 0; a < arows; a += p.abox) tma_load_2d(sA + a * p.r * 2, &tm_a, bar_ab, 0, k0 + a0 + a);
-      }
-    }
-    bool got = __all_sync(0xffffffffu, wait_bar(bar_ab, static_cast<uint32_t>(pass & 1), waiter));
-    if (kn > p.ka) got = __syncthreads_and(got) != 0;   // several passes: leave them together
-    ok = ok && got;
-    if (!ok) break;
-    if (xa_active) {
-      for (int kst = my_part; kst < arows / 16; kst += nsplit) {
-        const int kk = a0 + kst * 16;              // slice-relative contraction index
-        const uint32_t x0 = smem_u32(sX + g * xp + sk_xoff(kk) + 2 * c);
-        const uint32_t x8 = smem_u32(sX + (g + 8) * xp + sk_xoff(kk) + 2 * c);
-        uint32_t a[4] = {0u, 0u, 0u, 0u};
-        if (tok0) {
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[0]) : "r"(x0));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[2]) : "r"(x0 + 16));
-        }
-        if (tok1) {
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[1]) : "r"(x8));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[3]) : "r"(x8 + 16));
-        }
-        const uint32_t arow = smem_u32(sA + (kst * 16 + (lane & 15)) * p.r * 2);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int t8 = my_t8 + u * 8;
-          if (t8 < jt) {
-            uint32_t b0, b1;
-            ldmatrix_x2_trans(arow + t8 * 16, b0, b1);
-            mma_16816_bf16(xacc[u], a, b0, b1);
-          }
-        }
-      }
-    }
-  }
-  if (xa_active) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int t8 = my_t8 + u * 8;
-      if (t8 < jt) {
-        float *dst = (nsplit == 1) ? sXA + t8 * 8 : sSlot + warp * 128;
-        const int ld = (nsplit == 1) ? p.r : 8;
-        dst[g * ld + 2 * c] = xacc[u][0];
-        dst[g * ld + 2 * c + 1] = xacc[u][1];
-        dst[(g + 8) * ld + 2 * c] = xacc[u][2];
-        dst[(g + 8) * ld + 2 * c + 1] = xacc[u][3];
-      }
-    }
-  }
-
-  // ---- 3. main product over the macro-blocks
   const int ntiles = p.M > 8 ? 2 : 1;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  bool ok = true;
   const uint32_t codes_base = smem_u32(sm);
-  for (int mb = 0; mb < nmb && ok; ++mb) {
+  for (int mb = 0; mb < nmb; ++mb) {
     const uint32_t qa0 = qa[0], qb0 = qb[0];
     const float sa0 = sa[0], sb0 = sb[0];
 #pragma unroll
@@ -312,7 +248,7 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
     }
   }
 
-  // ---- 4. push the partial Y rows to the rank that finishes them: slot
+  // ---- 3. push the partial Y rows to the rank that finishes them: slot
   // [this rank][row within the owner's R][token] of the owner's receive buffer
   {
     const uint32_t recv = smem_u32(sRecv);
@@ -334,30 +270,14 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
       }
     }
   }
-  if (nsplit > 1) {
-    __syncthreads();
-    for (int i = tid; i < p.M * p.r; i += kSkThreads) {
-      const int t = i / p.r, j = i - t * p.r, t8 = j >> 3;
-      float v = 0.f;
-      for (int q = 0; q < nsplit; ++q) v += sSlot[(t8 * nsplit + q) * 128 + t * 8 + (j & 7)];
-      sXA[i] = v;
-    }
-  }
+  // XA comes from the XA kernel: wait for that grid (a no-op when launched plainly)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = tid; i < p.M * p.r; i += kSkThreads) sXA[i] = p.xa[i];
+  ok = __all_sync(0xffffffffu, wait_bar(bar_b, 0, waiter)) && ok;
 
-  // ---- 5. cluster reduction in rank order; rank q finishes rows [q R, (q+1) R)
+  // ---- 4. cluster barrier: every partial has landed in its owner's buffer; after
+  // it no CTA touches another's shared memory, so each may finish and leave
   if (C > 1) cluster_sync_all(); else __syncthreads();
-  float *sXAsum = sXA + 16 * p.r;
-  const uint32_t xa_base = smem_u32(sXA);
-  for (int i = tid; i < p.M * p.r; i += kSkThreads) {
-    float v = 0.f;
-#pragma unroll
-    for (int q = 0; q < C; ++q) v += ld_dsmem_f32(map_rank(xa_base + 4u * i, q));
-    sXAsum[i] = v;
-  }
-  __syncthreads();
-  if (p.XA_out && blockIdx.y == 0 && rank == 0) {
-    for (int i = tid; i < p.M * p.r; i += kSkThreads) p.XA_out[i] = sXAsum[i];
-  }
   for (int i = tid; i < R * p.M; i += kSkThreads) {
     const int tk = i / R, rr = i - tk * R;
     float v = 0.f;
@@ -365,19 +285,140 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
     for (int q = 0; q < C; ++q) v += sRecv[(q * R + rr) * 16 + tk];
     float lora = 0.f;
     for (int j = 0; j < p.r; ++j)
-      lora = fmaf(sXAsum[tk * p.r + j], __uint_as_float(static_cast<uint32_t>(sB[j * R + rr]) << 16), lora);
+      lora = fmaf(sXA[tk * p.r + j], __uint_as_float(static_cast<uint32_t>(sB[j * R + rr]) << 16), lora);
     const __nv_bfloat16 h = __float2bfloat16_rn(v + p.s * lora);
     p.Y[static_cast<int64_t>(tk) * p.N + w0 + static_cast<int>(rank) * R + rr] = *reinterpret_cast<const uint16_t *>(&h);
   }
-  // no CTA leaves while a peer may still read its shared memory; every value read
-  // from a peer has been consumed above, so the arrival needs no release
-  if (C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// XA = X A for few tokens: one cluster of kXaCluster CTAs, rank q takes rows
+// [q kx, (q+1) kx) of the contraction in chunks of `chunk` rows, each chunk of A
+// (contiguous) and of every token row of X fetched by one bulk copy; X rows on
+// the MMA's M (tokens), adapter columns on N.  Partials are summed by rank 0 in
+// rank order.
+constexpr int kXaCluster = 8;
+
+struct XaParams {
+  const uint16_t *X;   // [M, K] bf16
+  const uint16_t *A;   // [K, r] bf16
+  float *xa;           // [M, r] fp32
+  int M, K, r, kx;
+  int chunk;           // contraction rows per pass, a multiple of 16
+  uint64_t limit_ns;
+};
+
+inline int xa_chunk_rows(int r) { return r <= 64 ? 512 : 256; }
+inline int xa_smem_bytes(int r) {
+  const int ch = xa_chunk_rows(r);
+  return 16 * (ch + 8) * 2 + ch * r * 2 + 8 * 128 * 4 + 16 * r * 4 + 32;
+}
+
+__global__ void __launch_bounds__(256, 1) qlora_xa_kernel(const __grid_constant__ XaParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ __align__(128) uint8_t xa_smem[];
+  const int xpitch = p.chunk + 8;
+  uint16_t *sX = reinterpret_cast<uint16_t *>(xa_smem);                          // [16][xpitch]
+  uint8_t *sA = xa_smem + 16 * xpitch * 2;                                       // [chunk][r] dense
+  float *sSlot = reinterpret_cast<float *>(sA + p.chunk * p.r * 2);              // [8 warps][16][8]
+  float *sPart = sSlot + 8 * 128;                                                // [16][r]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sPart + 16 * p.r);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 1);
+  const Waiter waiter{abort_flag, p.limit_ns};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const uint32_t rank = cluster_ctarank();
+  const int k0 = min(p.K, static_cast<int>(rank) * p.kx), k1 = min(p.K, k0 + p.kx);
+  const bool tok0 = g < p.M, tok1 = g + 8 < p.M;
+  const int jt = p.r >> 3;
+  const int nsplit = jt >= 8 ? 1 : 8 / jt;
+  const int my_t8 = (jt >= 8) ? warp : warp / nsplit, my_part = (jt >= 8) ? 0 : warp % nsplit;
+  const bool active = (jt >= 8) || (warp < jt * nsplit);
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  bool ok = true;
+  int pass = 0;
+  for (int a0 = k0; a0 < k1; a0 += p.chunk, ++pass) {
+    const int rows = min(p.chunk, k1 - a0);
+    __syncthreads();                                // barrier init seen; the previous chunk consumed
+    if (tid == 0) {
+      const uint32_t arow_bytes = static_cast<uint32_t>(rows * 2);
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * p.r * 2) + arow_bytes * static_cast<uint32_t>(p.M));
+      bulk_load(sA, p.A + static_cast<int64_t>(a0) * p.r, static_cast<uint32_t>(rows * p.r * 2), bar);
+      for (int t = 0; t < p.M; ++t) bulk_load(sX + t * xpitch, p.X + static_cast<int64_t>(t) * p.K + a0, arow_bytes, bar);
+    }
+    const bool got = __syncthreads_and(wait_bar(bar, static_cast<uint32_t>(pass & 1), waiter)) != 0;
+    ok = ok && got;
+    if (!ok) break;
+    if (active) {
+      for (int kst = my_part; kst < rows / 16; kst += nsplit) {
+        const uint32_t x0 = smem_u32(sX + g * xpitch + kst * 16 + 2 * c);
+        const uint32_t x8 = smem_u32(sX + (g + 8) * xpitch + kst * 16 + 2 * c);
+        uint32_t a[4] = {0u, 0u, 0u, 0u};
+        if (tok0) {
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[0]) : "r"(x0));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[2]) : "r"(x0 + 16));
+        }
+        if (tok1) {
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[1]) : "r"(x8));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[3]) : "r"(x8 + 16));
+        }
+        const uint32_t arow = smem_u32(sA + (kst * 16 + (lane & 15)) * p.r * 2);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int t8 = my_t8 + u * 8;
+          if (t8 < jt) {
+            uint32_t b0, b1;
+            ldmatrix_x2_trans(arow + t8 * 16, b0, b1);
+            mma_16816_bf16(acc[u], a, b0, b1);
+          }
+        }
+      }
+    }
+  }
+  if (active) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int t8 = my_t8 + u * 8;
+      if (t8 < jt) {
+        float *dst = (nsplit == 1) ? sPart + t8 * 8 : sSlot + warp * 128;
+        const int ld = (nsplit == 1) ? p.r : 8;
+        dst[g * ld + 2 * c] = acc[u][0];
+        dst[g * ld + 2 * c + 1] = acc[u][1];
+        dst[(g + 8) * ld + 2 * c] = acc[u][2];
+        dst[(g + 8) * ld + 2 * c + 1] = acc[u][3];
+      }
+    }
+  }
+  if (nsplit > 1) {
+    __syncthreads();
+    for (int i = tid; i < p.M * p.r; i += 256) {
+      const int t = i / p.r, j = i - t * p.r, t8 = j >> 3;
+      float v = 0.f;
+      for (int q = 0; q < nsplit; ++q) v += sSlot[(t8 * nsplit + q) * 128 + t * 8 + (j & 7)];
+      sPart[i] = v;
+    }
+  }
+  cluster_sync_all();
+  if (rank == 0) {
+    const uint32_t base = smem_u32(sPart);
+    for (int i = tid; i < p.M * p.r; i += 256) {
+      float v = 0.f;
+#pragma unroll
+      for (int q = 0; q < kXaCluster; ++q) v += ld_dsmem_f32(map_rank(base + 4u * i, q));
+      p.xa[i] = v;
+    }
+  }
+  cluster_sync_all();   // the peers' partials stay until rank 0 has read them
 }
 
 // Shared-memory plan of one launch; false when nothing fits in `limit` bytes.
 struct SkinnyPlan {
-  int C, ks, ka, abox, xpitch;
-  int off_x, off_a, off_b, off_part, off_xa, off_slot, off_bar, smem;
+  int C, ks, xpitch;
+  int off_b, off_x, off_part, off_xa, off_bar, smem;
 };
 
 inline bool skinny_plan_for(int M, int K, int r, int C, int limit, SkinnyPlan &pl) {
@@ -388,27 +429,16 @@ inline bool skinny_plan_for(int M, int K, int r, int C, int limit, SkinnyPlan &p
   const int xbase = pl.ks + pl.ks / 16;
   pl.xpitch = xbase + (((16 - xbase) % 64) + 64) % 64;
   const int nbars = pl.ks / kSkMacro + 1;
-  const int fixed = 1024 + (pl.ks / kSkMacro) * kSkBoxBytes + up16(M * pl.xpitch * 2) +
-                    ((r * (kSkRows / C) * 2 + 127) & ~127) + kSkRows * 16 * 4 + 2 * 16 * r * 4 + 8 * 128 * 4 +
-                    8 * nbars + 16;
-  int ka = pl.ks;
-  while (ka >= 16 && fixed + ka * 2 * r > limit) ka = (ka / 2) & ~15;
-  if (ka < 16) return false;
-  pl.abox = ka < 256 ? ka : 256;
-  ka = ka / pl.abox * pl.abox;
-  pl.ka = ka;
-  // TMA destinations first: the code boxes (1024-byte aligned for the 128B
-  // swizzle), then A and B, whose boxes need 128-byte aligned shared memory
+  // bulk-copy destinations first: the code boxes (1024-byte aligned for the
+  // 128B swizzle), then B (128-byte aligned)
   int off = (pl.ks / kSkMacro) * kSkBoxBytes;
-  pl.off_a = off;    off += ka * 2 * r;
   pl.off_b = off;    off += (r * (kSkRows / C) * 2 + 127) & ~127;
   pl.off_x = off;    off += up16(M * pl.xpitch * 2);
   pl.off_part = off; off += kSkRows * 16 * 4;
-  pl.off_xa = off;   off += 2 * 16 * r * 4;
-  pl.off_slot = off; off += 8 * 128 * 4;
+  pl.off_xa = off;   off += up16(M * r * 4);
   pl.off_bar = off;  off += 8 * nbars + 16;
   pl.smem = off + 1024;                          // slack for aligning the base to 1024 bytes
-  if ((pl.off_a & 127) || (pl.off_b & 127) || ((pl.abox * 2 * r) & 127)) return false;
+  if (pl.off_b & 127) return false;
   return pl.smem <= limit;
 }
 
