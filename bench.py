@@ -53,12 +53,22 @@ def peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def source_hash():
-    h = hashlib.sha256()
+def source_hash(kernel_key):
+    """Hash of the code that defines one kernel's launch: its own header, the
+    shared device helpers, and the host function that configures the launch."""
     csrc = os.path.join(ROOT, "bit_nf4_quantized_19_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files, launcher = {
+        "qlora_gemm_kernel": (["gemm_kernel.cuh", "common.cuh"], "qlora_status launch_gemm("),
+        "qlora_skinny_kernel": (["skinny_kernel.cuh", "common.cuh"], "qlora_status launch_skinny("),
+    }[kernel_key]
+    h = hashlib.sha256()
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "qlora_nf4.cu")) as fh:
+        text = fh.read()
+    i = text.find(launcher)
+    h.update(text[i:text.find("\n}\n", i)].encode() if i >= 0 else b"")
     return h.hexdigest()[:16]
 
 
@@ -69,7 +79,7 @@ def traffic_for(kernel_key):
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
         e = t.get(kernel_key)
-        if e and e.get("source_hash") == source_hash():
+        if e and e.get("source_hash") == source_hash(kernel_key):
             return e.get("bytes_per_launch")
     except Exception:
         pass
