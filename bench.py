@@ -221,9 +221,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="M,N,K: small profiling case (two fwd+bwd of one projection), no JSON")
+    ap.add_argument("--quant-case", type=int, default=None,
+                    help="N: profiling case, quantize + dequant of N heavy-tailed values twice, no JSON")
     args = ap.parse_args()
     if args.case:
         return profile_case(*[int(v) for v in args.case.split(",")])
+    if args.quant_case:
+        return profile_quant_case(args.quant_case)
     args.warmup = max(3, args.warmup)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -339,19 +343,46 @@ def main():
             "avg_launch_ms": gemm_ms / max(1, gemm_launches),
             "traffic": traffic_for("qlora_gemm_kernel")}
 
-    # ---- end to end through the public API: pinned host inputs -> device -> grads back
+    # ---- end to end through the public API: pinned host inputs -> device -> grads back.
+    # As a data loader would, the next step's inputs are uploaded (on their own stream,
+    # into the other of two device buffers) while the current step computes; every
+    # upload and every read-back of the gradients lies inside the timed region.
     e2e_steps = max(3, min(args.steps, 30))
     h2d = sum(L["hX"].numel() * 2 + L["hdY"].numel() * 2 for L in layers)
     d2h = flat_host.numel() * 4
+    xfer = torch.cuda.Stream(device=dev)
+    bufs = [[(L["X"], L["dY"]) for L in layers],
+            [(torch.empty_like(L["X"]), torch.empty_like(L["dY"])) for L in layers]]
+    uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def upload(b):
+        xfer.wait_event(consumed[b])          # the step that last read buffer b is done
+        with torch.cuda.stream(xfer):
+            for (X, dY), L in zip(bufs[b], layers):
+                X.copy_(L["hX"], non_blocking=True)
+                dY.copy_(L["hdY"], non_blocking=True)
+        uploaded[b].record(xfer)
+
+    def step_on(b):
+        stream.wait_event(uploaded[b])
+        for (X, dY), L in zip(bufs[b], layers):
+            q.linear_fwd(X, L["Wq"], L["A"], L["B"], L["s"], workspace=L["ws"], Y=L["Y"], XA=L["XA"])
+            q.linear_bwd(dY, X, L["XA"], L["Wq"], L["A"], L["B"], L["s"],
+                         workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
+        bucket.allreduce_()
+        consumed[b].record(stream)
+
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
+    xfer.wait_event(e0)
+    upload(0)
     for i in range(e2e_steps):
-        for L in layers:
-            L["X"].copy_(L["hX"], non_blocking=True)
-            L["dY"].copy_(L["hdY"], non_blocking=True)
-        step()
+        if i + 1 < e2e_steps:
+            upload((i + 1) % 2)
+        step_on(i % 2)
         flat_host.copy_(flat_grads, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -362,7 +393,7 @@ def main():
         e2e_ms = float(t.item())
     e2e = {"value": world * flops_per_step_rank * e2e_steps / (e2e_ms * 1e-3) / 1e12,
            "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "steps": e2e_steps}
+           "steps": e2e_steps, "uploads": "next step's inputs overlap the current step (two buffers)"}
 
     # ---- HBM-bound subpaths (quantize / dequant of 1e9 values, skinny forward)
     subpaths = None
@@ -425,20 +456,41 @@ def profile_case(M, N, K, r=RANK_R):
     return 0 if code == 0 else 1
 
 
+def heavy_tail_device(torch, dev, n, seed=0):
+    """n bf16 values ~ N(0, 0.02), each scaled by 8 with probability 1e-3 (seeded, on the device)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    W = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    chunk = 1 << 26
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        z = torch.randn(m, generator=g, device=dev, dtype=torch.float32) * 0.02
+        z[torch.rand(m, generator=g, device=dev) < 1e-3] *= 8.0
+        W[i:i + m] = z.to(torch.bfloat16)
+    return W
+
+
+def profile_quant_case(n):
+    """Quantize + dequant of n heavy-tailed values, twice, through the public API;
+    the case that the quantize/dequant ncu captures under profiles/ use."""
+    import torch
+    import bit_nf4_quantized_19_b200 as q
+    W = heavy_tail_device(torch, torch.device("cuda"), n)
+    out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    Wq = q.nf4_quantize(W.view(1, n))
+    for _ in range(2):
+        q.nf4_quantize(W.view(1, n), out=Wq)
+        q.nf4_dequant(Wq, out.view(1, n))
+    torch.cuda.synchronize()
+    code, flags = q.device_status()
+    print("quant case", n, "status", code, flags)
+    return 0 if code == 0 else 1
+
+
 def hbm_subpaths(q, torch, dev, stream, P, flush):
     out = {}
     # 1e9-value heavy-tailed tensor, generated on the device (seeded)
-    g = torch.Generator(device=dev)
-    g.manual_seed(0)
-    W = torch.empty(BIG_N, dtype=torch.bfloat16, device=dev)
-    chunk = 1 << 26
-    for i in range(0, BIG_N, chunk):
-        n = min(chunk, BIG_N - i)
-        z = torch.randn(n, generator=g, device=dev, dtype=torch.float32) * 0.02
-        m = torch.rand(n, generator=g, device=dev) < 1e-3
-        z[m] *= 8.0
-        W[i:i + n] = z.to(torch.bfloat16)
-    del z, m
+    W = heavy_tail_device(torch, dev, BIG_N)
     Wq = q.nf4_quantize(W.view(1, BIG_N))
     out_bf = torch.empty(BIG_N, dtype=torch.bfloat16, device=dev)
     q.nf4_dequant(Wq, out_bf.view(1, BIG_N))

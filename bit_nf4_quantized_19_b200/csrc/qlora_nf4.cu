@@ -69,7 +69,9 @@ qlora_status device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if (cudaFuncSetAttribute(qlora_xa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(qlora_xa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              xa_smem_bytes(64) > xa_smem_bytes(128) ? xa_smem_bytes(64) : xa_smem_bytes(128)) !=
             cudaSuccess ||
         set_skinny_attrs<1>() != cudaSuccess || set_skinny_attrs<2>() != cudaSuccess ||
@@ -580,13 +582,19 @@ qlora_status qlora_nf4_quantize(const uint16_t *W, int64_t rows, int64_t cols,
   const Nf4Tables &T = nf4_tables();
   if (!T.ok) return QLORA_ERR_DEVICE_CHECK;
   QuantTables tab;
-  std::memcpy(tab.bins, T.bins, sizeof(tab.bins));
+  for (int i = 0; i < kQuantBins256; ++i) {
+    tab.bins[i].t = 2.0f;                         // inert: reachable only from non-finite blocks
+    tab.bins[i].c = 0;
+  }
+  for (int j = -32; j <= 32; ++j) tab.bins[j + 32] = T.bins[j & (kQuantBins - 1)];
   std::memcpy(tab.rcp, T.rcp, sizeof(tab.rcp));
   const int64_t n = rows * cols;
   const int64_t groups = (n + kGroupElems - 1) / kGroupElems;
   if (groups > 0x7FFFFFFFll) return QLORA_ERR_UNSUPPORTED_SHAPE;
   LaunchTimer lt(QLORA_K_QUANTIZE, stream);
-  nf4_quantize_kernel<<<static_cast<unsigned>(groups), 256, 0, stream>>>(W, n, out->codes, out->q8,
+  const int64_t grid = groups < static_cast<int64_t>(d->sms) * kQuantCtasPerSm ? groups
+                                                                                : static_cast<int64_t>(d->sms) * kQuantCtasPerSm;
+  nf4_quantize_kernel<<<static_cast<unsigned>(grid > 0 ? grid : 1), 256, kQuantSmemBytes, stream>>>(W, n, out->codes, out->q8,
                                                                          out->step, tab);
   return cuda_status(cudaGetLastError());
 }

@@ -12,17 +12,22 @@ constexpr int kBlock = 64;                 // values per first-level block
 constexpr int kGroup = 256;                // blocks per second-level constant
 constexpr int kGroupElems = kBlock * kGroup;
 
+// Bin table of the quantize kernel, indexed by the low byte of 32 xn + 32 + 1.5*2^23:
+// entries 0..64 are the bins round(32 xn) = -32..32; the rest are reachable only from
+// a non-finite block and hold an inert bin (t = 2, c = 0).
+constexpr int kQuantBins256 = 256;
 struct QuantTables {
-  QuantBin bins[kQuantBins];   // indexed by round(32 * xn) mod 128
+  QuantBin bins[kQuantBins256];
   float rcp[128];              // RN32(1 / (1 + k/128)): reciprocals of the bf16 mantissas
 };
 struct Levels {
   float v[16];
 };
 
-// One CTA per group of 256 blocks (16384 values); 256 threads; 8 threads per
-// block, each owning 8 consecutive values (one 16-byte load), 32 blocks per pass,
-// 8 passes.  All eight 16-byte loads are issued before any arithmetic.
+// Persistent CTAs (three per SM), each looping over groups of 256 blocks (16384
+// values); 256 threads; 8 threads per block, each owning 8 consecutive values (one
+// 16-byte load), 32 blocks per pass, 8 passes.  All eight 16-byte loads of a group
+// are issued before any arithmetic.
 //   absmax: max |w| within the thread, then an xor-shuffle over the 8 lanes;
 //   xn:     RN32(w / a_b).  For 2^-64 <= a_b <= 2^64 (every realistic block) the
 //           division is Markstein's FMA correction of w * RN32(1/a_b), where
@@ -30,34 +35,56 @@ struct Levels {
 //           a_b is a bf16 value; outside that range, IEEE division.  An exhaustive
 //           host check over all bf16 pairs of the fast range shows both give the
 //           same code for every input (tests/csrc/division_check.c);
-//   code:   bin j = round(32 xn) (exact, from the sum 32 xn + 1.5*2^23), then
-//           code = bins[j].c + (xn > bins[j].t): the number of decision thresholds
-//           below xn, i.e. the nearest level with ties to the lower index;
-//   pack:   8 codes -> one 32-bit word (element 2j in the low nibble of byte j);
+//   code:   bin j = round(32 xn) (exact, the low byte of 32 xn + 32 + 1.5*2^23 is
+//           j + 32), then code = bins[j].c + (xn > bins[j].t): the number of decision
+//           thresholds below xn, i.e. the nearest level with ties to the lower index.
+//           Every lane reads its own copy of the bin table (entry i of lane l at byte
+//           256 i + 8 l, one byte permute away from the sum), so the data-dependent
+//           lookups never conflict on a bank;
+//   pack:   8 codes -> one 32-bit word (element 2j in the low nibble of byte j),
+//           accumulated as word = 16 word + code from the last element down;
 //   double quant (after all passes): c_g = max a_b over the group,
 //           step = RN32(c_g / 255), q8 = min(255, rint(RN32(a_b / step))).
-__global__ void __launch_bounds__(256, 3) nf4_quantize_kernel(
-    const uint16_t *__restrict__ W, int64_t n, uint8_t *__restrict__ codes,
-    uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab) {
-  __shared__ QuantBin bins[kQuantBins];
-  __shared__ float rcp[128];
-  __shared__ float amax[kGroup];
-  __shared__ float wmax[8];
-  const int tid = threadIdx.x;
-  if (tid < kQuantBins) bins[tid] = tab.bins[tid];
-  if (tid < 128) rcp[tid] = tab.rcp[tid];
+// Markstein's quotient (P. Markstein, "IA-64 and Elementary Functions", 2000) for
+// two values at once with the packed fp32 FMA of sm_100 (each lane an IEEE fp32
+// operation with a single rounding, subnormals kept): q0 = w*y, r = fma(q0, -a, w),
+// xn = fma(r, y, q0); also f = fma(xn, 32, 1.5*2^23 + 32), whose low byte is
+// round(32 xn) + 32 for |xn| <= 1.
+QDEV void quotient_x2(float w0, float w1, float y, float neg_a, float &xn0, float &xn1, float &f0,
+                      float &f1) {
+  asm("{\n\t.reg .b64 w, yy, na, q, r, x, k, m, f;\n\t"
+      "mov.b64 w, {%4, %5};\n\t"
+      "mov.b64 yy, {%6, %6};\n\t"
+      "mov.b64 na, {%7, %7};\n\t"
+      "mov.b64 k, {%8, %8};\n\t"
+      "mov.b64 m, {%9, %9};\n\t"
+      "mul.rn.f32x2 q, w, yy;\n\t"
+      "fma.rn.f32x2 r, q, na, w;\n\t"
+      "fma.rn.f32x2 x, r, yy, q;\n\t"
+      "fma.rn.f32x2 f, x, k, m;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t"
+      "mov.b64 {%2, %3}, f;\n\t}"
+      : "=f"(xn0), "=f"(xn1), "=f"(f0), "=f"(f1)
+      : "f"(w0), "f"(w1), "f"(y), "f"(neg_a), "f"(32.0f), "f"(12582944.0f));
+}
 
-  const int64_t g = blockIdx.x;
-  const int64_t gbase = g * kGroupElems;
-  const int sub = tid & 7;
-  const int bl = tid >> 3;
+// max of two bf16x2 words, lane by lane, NaN-propagating
+QDEV uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 
-  uint4 v[8];
+// The eight 16-byte loads of one thread for one group (pass p: block 32 p + bl,
+// values 8 sub .. 8 sub + 7); WHOLE = the group lies entirely inside the tensor.
+template <bool WHOLE>
+QDEV void quant_load(const uint16_t *__restrict__ W, int64_t n, int64_t gbase, int bl, int sub, uint4 (&v)[8]) {
+  const uint16_t *base = W + gbase + bl * kBlock + sub * 8;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     const int64_t e = gbase + static_cast<int64_t>(p * 32 + bl) * kBlock + sub * 8;
-    if (e + 8 <= n) {
-      v[p] = ld_global_nc_v4(W + e);
+    if (WHOLE || e + 8 <= n) {
+      v[p] = ld_global_nc_v4(base + p * 32 * kBlock);
     } else {
       uint32_t t[4] = {0, 0, 0, 0};
       for (int j = 0; j < 8; ++j)
@@ -65,9 +92,34 @@ __global__ void __launch_bounds__(256, 3) nf4_quantize_kernel(
       v[p] = make_uint4(t[0], t[1], t[2], t[3]);
     }
   }
-  __syncthreads();
+}
 
-  bool nonfinite = false;
+// Codes of one group.  The eight block absmaxes come first, on the packed bf16
+// words (|w| is w with the sign bits cleared; NaN propagates), two passes per
+// shuffle; one warp vote then picks the path for the whole group.
+template <bool WHOLE>
+QDEV void quant_compute(const uint4 (&v)[8], int64_t n, int64_t gbase, int bl, int sub, const float *rcp,
+                        const uint8_t *bins_bytes, uint32_t lane8, uint8_t *__restrict__ codes,
+                        float *amax, bool &nonfinite) {
+  float am[8];
+#pragma unroll
+  for (int p = 0; p < 8; p += 2) {
+    uint32_t m0 = bmax2(bmax2(v[p].x & 0x7FFF7FFFu, v[p].y & 0x7FFF7FFFu), bmax2(v[p].z & 0x7FFF7FFFu, v[p].w & 0x7FFF7FFFu));
+    uint32_t m1 = bmax2(bmax2(v[p + 1].x & 0x7FFF7FFFu, v[p + 1].y & 0x7FFF7FFFu),
+                        bmax2(v[p + 1].z & 0x7FFF7FFFu, v[p + 1].w & 0x7FFF7FFFu));
+    // low half: pass p, high half: pass p + 1
+    uint32_t mm = bmax2(prmt(m0, m1, 0x5410u), prmt(m0, m1, 0x7632u));
+    mm = bmax2(mm, __shfl_xor_sync(0xffffffffu, mm, 1));
+    mm = bmax2(mm, __shfl_xor_sync(0xffffffffu, mm, 2));
+    mm = bmax2(mm, __shfl_xor_sync(0xffffffffu, mm, 4));
+    am[p] = __uint_as_float(mm << 16);
+    am[p + 1] = __uint_as_float(mm & 0xFFFF0000u);
+  }
+  bool fast = true;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) fast = fast && (am[p] >= 0x1p-64f) && (am[p] <= 0x1p64f);
+  const bool group_fast = __all_sync(0xffffffffu, fast);
+  uint8_t *cbase = codes + ((gbase + bl * kBlock + sub * 8) >> 1);
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     const int64_t e = gbase + static_cast<int64_t>(p * 32 + bl) * kBlock + sub * 8;
@@ -75,51 +127,48 @@ __global__ void __launch_bounds__(256, 3) nf4_quantize_kernel(
     float w[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      w[2 * j] = bf16_lo(wd[j]);
+      w[2 * j] = __uint_as_float(wd[j] * 65536u);
       w[2 * j + 1] = bf16_hi(wd[j]);
     }
-    float am = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(w[j]));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
-    if (!(am <= 3.402823466e38f)) nonfinite = true;
-    const bool fast = (am >= 0x1p-64f) && (am <= 0x1p64f);
-    // RN32(1/am) = RN32(1/m) * 2^-e for am = m * 2^e (m has 7 fraction bits)
-    const uint32_t ab = __float_as_uint(am);
+    const float a_b = am[p];
+    // RN32(1/a_b) = RN32(1/m) * 2^-e for a_b = m * 2^e (m has 7 fraction bits)
+    const uint32_t ab = __float_as_uint(a_b);
     const int ex = static_cast<int>((ab >> 23) & 0xFFu) - 127;
     const float y = __uint_as_float(__float_as_uint(rcp[(ab >> 16) & 127u]) - (static_cast<uint32_t>(ex) << 23));
     uint32_t word = 0;
-    if (__all_sync(0xffffffffu, fast)) {
+    if (group_fast) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float q0 = __fmul_rn(w[j], y);
-        const float r = __fmaf_rn(-q0, am, w[j]);
-        const float xn = __fmaf_rn(r, y, q0);
-        const float f = __fmaf_rn(xn, 32.0f, 12582912.0f);
-        const QuantBin b = bins[__float_as_uint(f) & (kQuantBins - 1)];
-        word |= static_cast<uint32_t>(b.c + (xn > b.t ? 1 : 0)) << (4 * j);
+      for (int j = 6; j >= 0; j -= 2) {
+        float xa, xb, fa, fb;
+        quotient_x2(w[j], w[j + 1], y, -a_b, xa, xb, fa, fb);
+        const uint2 tb = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(fb), lane8, 0x5504u));
+        const uint2 ta = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(fa), lane8, 0x5504u));
+        // xn > t exactly when t - xn is negative (both finite; no threshold is zero,
+        // so the difference is never a negative zero): its sign bit is the increment
+        word = word * 16u + tb.y + (__float_as_uint(__fsub_rn(__uint_as_float(tb.x), xb)) >> 31);
+        word = word * 16u + ta.y + (__float_as_uint(__fsub_rn(__uint_as_float(ta.x), xa)) >> 31);
       }
     } else {
-      const float a = (am > 0.f) ? am : 1.0f;
+      const bool fast_b = (a_b >= 0x1p-64f) && (a_b <= 0x1p64f);
+      if (!(a_b <= 3.402823466e38f)) nonfinite = true;     // inf or NaN somewhere in the block
+      const float a = (a_b > 0.f) ? a_b : 1.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 7; j >= 0; --j) {
         float xn;
-        if (fast) {
+        if (fast_b) {
           const float q0 = __fmul_rn(w[j], y);
-          const float r = __fmaf_rn(-q0, am, w[j]);
+          const float r = __fmaf_rn(-q0, a_b, w[j]);
           xn = __fmaf_rn(r, y, q0);
         } else {
           xn = __fdiv_rn(w[j], a);
         }
-        const float f = __fmaf_rn(xn, 32.0f, 12582912.0f);
-        const QuantBin b = bins[__float_as_uint(f) & (kQuantBins - 1)];
-        word |= static_cast<uint32_t>(b.c + (xn > b.t ? 1 : 0)) << (4 * j);
+        const float f = __fmaf_rn(xn, 32.0f, 12582944.0f);
+        const uint2 t = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(f), lane8, 0x5504u));
+        word = word * 16u + t.y + (xn > __uint_as_float(t.x) ? 1u : 0u);
       }
     }
-    if (e + 8 <= n) {
-      *reinterpret_cast<uint32_t *>(codes + (e >> 1)) = word;
+    if (WHOLE || e + 8 <= n) {
+      *reinterpret_cast<uint32_t *>(cbase + p * 32 * kBlock / 2) = word;
     } else if (e < n) {
       const int valid = static_cast<int>(n - e);           // 1..7
       const uint32_t keep = (1u << (4 * valid)) - 1u;      // zero the nibbles past n
@@ -127,30 +176,69 @@ __global__ void __launch_bounds__(256, 3) nf4_quantize_kernel(
       const int nbytes = (valid + 1) >> 1;
       for (int j = 0; j < nbytes; ++j) codes[(e >> 1) + j] = static_cast<uint8_t>(word >> (8 * j));
     }
-    if (sub == 0) amax[p * 32 + bl] = am;
+    if (sub == 0) amax[p * 32 + bl] = a_b;
+  }
+}
+
+constexpr int kQuantCtasPerSm = 3;
+constexpr int kQuantSmemBytes = kQuantBins256 * 32 * 8 + (128 + 256 + 8) * 4;
+
+__global__ void __launch_bounds__(256, kQuantCtasPerSm) nf4_quantize_kernel(
+    const uint16_t *__restrict__ W, int64_t n, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  uint2 *bins = reinterpret_cast<uint2 *>(qsm);                          // [256 entries][32 lanes]: (t bits, c)
+  float *rcp = reinterpret_cast<float *>(qsm + kQuantBins256 * 32 * 8);  // [128]
+  float *amax = rcp + 128;                                               // [256]
+  float *wmax = amax + kGroup;                                           // [8]
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < kQuantBins256 * 32; i += 256) {
+    const QuantBin e = tab.bins[i >> 5];
+    bins[i] = make_uint2(__float_as_uint(e.t), static_cast<uint32_t>(e.c));
+  }
+  if (tid < 128) rcp[tid] = tab.rcp[tid];
+  const uint32_t lane8 = 8u * static_cast<uint32_t>(lane);
+  const uint8_t *bins_bytes = qsm;
+  const int sub = tid & 7;
+  const int bl = tid >> 3;
+  const int64_t ngroups = (n + kGroupElems - 1) / kGroupElems;
+  const int64_t nblocks = (n + kBlock - 1) / kBlock;
+  bool nonfinite = false;
+
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const int64_t gbase = g * kGroupElems;
+    uint4 v[8];
+    if (gbase + kGroupElems <= n) {
+      quant_load<true>(W, n, gbase, bl, sub, v);
+      __syncthreads();   // tables filled; the previous group's amax and wmax consumed
+      quant_compute<true>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
+    } else {
+      quant_load<false>(W, n, gbase, bl, sub, v);
+      __syncthreads();
+      quant_compute<false>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
+    }
+    __syncthreads();
+
+    // second level: one constant per group
+    const int64_t b = g * kGroup + tid;
+    const float a = (b < nblocks) ? amax[tid] : 0.f;
+    float m = a;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) wmax[tid >> 5] = m;
+    __syncthreads();
+    float c = wmax[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) c = fmaxf(c, wmax[i]);
+    const float st = (c > 0.f) ? __fdiv_rn(c, 255.0f) : 0.f;
+    if (b < nblocks) {
+      int q = 0;
+      if (c > 0.f) q = min(255, __float2int_rn(__fdiv_rn(a, st)));
+      q8[b] = static_cast<uint8_t>(q);
+    }
+    if (tid == 0) step[g] = st;
   }
   if (nonfinite && sub == 0) atomicOr(&g_device_status, kStatNonFinite);
-  __syncthreads();
-
-  // second level: one constant per group
-  const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  const int64_t b = g * kGroup + tid;
-  const float a = (b < nblocks) ? amax[tid] : 0.f;
-  float m = a;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((tid & 31) == 0) wmax[tid >> 5] = m;
-  __syncthreads();
-  float c = wmax[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) c = fmaxf(c, wmax[i]);
-  const float st = (c > 0.f) ? __fdiv_rn(c, 255.0f) : 0.f;
-  if (b < nblocks) {
-    int q = 0;
-    if (c > 0.f) q = min(255, __float2int_rn(__fdiv_rn(a, st)));
-    q8[b] = static_cast<uint8_t>(q);
-  }
-  if (tid == 0) step[g] = st;
 }
 
 // Standalone dequant: 16 values per thread per iteration (8 bytes of codes in,

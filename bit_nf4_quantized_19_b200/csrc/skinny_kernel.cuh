@@ -78,14 +78,6 @@ QDEV float ld_dsmem_f32(uint32_t addr) {
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
-QDEV uint2 ld_shared_v2(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-QDEV void st_shared_v2(uint32_t a, uint32_t x, uint32_t y) {
-  asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(x), "r"(y) : "memory");
-}
 // Two transposed 8x8 bf16 tiles: lanes 0-7 address the rows of the first, 8-15
 // of the second; lane 4g+c receives rows 2c, 2c+1 of column g of each.
 QDEV void ldmatrix_x2_trans(uint32_t addr, uint32_t &b0, uint32_t &b1) {

@@ -85,9 +85,10 @@ def test_quantize_exhaustive_bf16_magnitudes(q):
     _check_quant(q, bits, 1, bits.size)
 
 
-def test_nonfinite_input_sets_device_status(q):
+@pytest.mark.parametrize("bad", [0x7F80, 0xFF80, 0x7FC0, 0xFFC1])   # +inf, -inf, quiet NaN, negative NaN
+def test_nonfinite_input_sets_device_status(q, bad):
     bits = normal_bf16(0, "nonfinite", (1, 4096), 0.02)
-    bits[0, 100] = 0x7F80   # +inf
+    bits[0, 100] = bad
     Wq, code, flags = _gpu_quant(q, bits, 1, 4096)
     assert code == 6 and (flags & 2)
     code2, flags2 = q.device_status()
