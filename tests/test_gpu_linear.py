@@ -115,6 +115,17 @@ def test_linear_llama7b_shapes_sampled_rows(q, N, K):
     _check(p, got, rows=rows)
 
 
+@pytest.mark.parametrize("N,K", [(8192, 8192), (22016, 8192), (8192, 22016)])
+def test_linear_llama65b_shapes_sampled_rows(q, N, K):
+    """The 8192-token LLaMA-65B-shaped projections (r = 64, alpha = 16, W ~ N(0, 0.015))
+    at full size; Y and dX on 48 seeded token rows (including the first and last),
+    XA, dA and dB in full."""
+    p = linear_problem(8192, N, K, 64, 16.0, 0.015, seed=0)
+    got = _run(q, p)
+    rows = np.unique(np.concatenate([[0, 8191], np.random.default_rng(6).integers(0, 8192, 46)]))
+    _check(p, got, rows=rows)
+
+
 @pytest.mark.parametrize("N,K", [(256, 384), (384, 256), (128, 1024)])
 def test_gemm_dequant_bit_exact_one_hot(q, N, K):
     """With X = I (K one-hot tokens) and A = 0 every output of the forward is a
