@@ -70,8 +70,8 @@ SIGNATURES = {
     "qlora_profile_read": (_int, [_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float)]),
 }
 
-KERNEL_KINDS = ["quantize", "dequant", "expand_scales", "project", "gemm_fwd", "gemm_dx",
-                "grad_partial", "grad_reduce", "skinny"]
+KERNEL_KINDS = ["quantize", "dequant", "prep", "project", "gemm_fwd", "gemm_dx",
+                "grad", "unused", "skinny"]
 PROFILE_CAP = 4096
 
 _LIB = None

@@ -6,9 +6,12 @@
 // with nn = r (rounded up to 16) or 2r (bf16 hi|lo halves of an fp32
 // operand), so it is bound by reading the bf16 activation (X or dY) once.
 //
-// One CTA computes a 128-row tile over one split of the contraction and writes
-// an fp32 partial tile; a separate reduction sums the splits in a fixed order
-// (deterministic).  The activation side is the MMA's A operand:
+// One CTA computes a 128-row tile over one split of the contraction.  The splits
+// of a tile form a thread-block cluster (at most 8): each CTA stages its fp32
+// partial tile in shared memory (reusing its operand ring, idle once the last
+// MMA has committed), and rank q then sums rows [q R, (q+1) R) over the cluster
+// in rank order through distributed shared memory (deterministic, no global
+// scratch) and writes the final outputs.  The activation side is the MMA's A operand:
 //   K-major  (projections): Act = X / dY tile [128 tokens x 64 c], TMA box {64, 128}
 //   MN-major (gradients):   Act^T tile [128 features x 64 tokens] from X / dY
 //                           [tokens, features]: two TMA boxes {64 features, 64 tokens}
@@ -30,12 +33,29 @@ struct LoraMmaParams {
   int stages_per_split;
   int num_stages;        // smem ring depth
   uint32_t tmem_cols;    // power of two >= max(32, nn)
-  float *partial;        // [splits][rows][nn]
+  int splits;            // cluster size along the contraction
+  int grad;              // 0: projection outputs, 1: gradient outputs
+  int r;
+  float s;
+  // projection: out [rows, r] fp32, hl [rows, 2r] and/or hlT [2r, ldT] bf16 hi|lo of s*out
+  // gradient:   out = sum of the hi and lo halves; layout 0 out[row][j], 1 out[j][row]
+  float *out;
+  uint16_t *hl;
+  uint16_t *hlT;
+  int ldT;
+  int layout;
   uint64_t limit_ns;
 };
 
 inline int lora_mma_smem_bytes(int nn, int stages) {
   return 1024 + stages * (kLmABytes + nn * 128) + 256;
+}
+
+QDEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+  hi = *reinterpret_cast<const uint16_t *>(&h);
+  lo = *reinterpret_cast<const uint16_t *>(&l);
 }
 
 template <bool A_MN>
@@ -125,13 +145,14 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     (void)ok;
     mma_commit(done);   // also drains every issued MMA before TMEM is released
   } else if (warp >= 4) {
+    // TMEM -> this CTA's partial tile in shared memory (the operand ring is idle now)
     const int q = warp & 3;
-    const int row = row0 + q * 32 + lane;
+    const int rl = q * 32 + lane;
     volatile int no_abort = 0;
     const Waiter dw{&no_abort, p.limit_ns};
     const bool got = __all_sync(0xffffffffu, wait_bar(done, 0, dw) ? 1 : 0);
     tc_fence_after();
-    float *dst = p.partial + (static_cast<int64_t>(split) * p.rows + row) * p.nn;
+    float *dst = reinterpret_cast<float *>(smem) + rl * p.nn;
     for (int c = 0; c < p.nn; c += 16) {
       uint32_t v[16];
       asm volatile(
@@ -142,20 +163,13 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
           : "r"(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c)));
       tmem_wait_ld();
-      if (row < p.rows) {
-        float4 *d4 = reinterpret_cast<float4 *>(dst + c);
+      const bool keep = got && nst > 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float4 o;
-          if (got && nst > 0) {
-            o = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          } else {
-            o = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-          d4[j] = o;
-        }
-      }
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4 *>(dst + c + 4 * j) =
+            keep ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   tc_fence_before();
@@ -165,6 +179,46 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
+
+  // ---- cluster reduction: rank q finishes rows [q R, (q+1) R) of the tile
+  cluster_sync_all();
+  {
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int R = (kLmRows + p.splits - 1) / p.splits;
+    const int r0 = rank * R, r1 = min(kLmRows, r0 + R);
+    const int nr = max(0, r1 - r0);
+    const uint32_t base = smem_u32(smem);
+    for (int i = tid; i < nr * p.r; i += kLmThreads) {
+      int rr, j;
+      if (p.grad && p.layout == 0) { rr = i / p.r; j = i - rr * p.r; }   // j fastest: out[row][j]
+      else { j = i / nr; rr = i - j * nr; }                               // row fastest
+      const int rl = r0 + rr, row = row0 + rl;
+      if (row >= p.rows) continue;
+      const uint32_t a = base + 4u * static_cast<uint32_t>(rl * p.nn + j);
+      float v = 0.f;
+      if (p.grad) {
+        const uint32_t b = a + 4u * static_cast<uint32_t>(p.r);
+        for (int qq = 0; qq < p.splits; ++qq)
+          v += ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) + ld_dsmem_f32(map_rank(b, static_cast<uint32_t>(qq)));
+        if (p.layout == 0) p.out[static_cast<int64_t>(row) * p.r + j] = v;
+        else p.out[static_cast<int64_t>(j) * p.rows + row] = v;
+      } else {
+        for (int qq = 0; qq < p.splits; ++qq) v += ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq)));
+        if (p.out) p.out[static_cast<int64_t>(row) * p.r + j] = v;
+        uint16_t h, l;
+        split_hilo(p.s * v, h, l);
+        if (p.hl) {
+          p.hl[static_cast<int64_t>(row) * 2 * p.r + j] = h;
+          p.hl[static_cast<int64_t>(row) * 2 * p.r + p.r + j] = l;
+        }
+        if (p.hlT) {
+          p.hlT[static_cast<int64_t>(j) * p.ldT + row] = h;
+          p.hlT[static_cast<int64_t>(p.r + j) * p.ldT + row] = l;
+        }
+      }
+    }
+  }
+  cluster_sync_all();   // no CTA leaves while a peer may still read its partial tile
 }
 
 // ---------------------------------------------------------------- helpers around it
@@ -176,42 +230,6 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__r
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t j = i / K, k = i - j * K;
     AT[i] = A[k * r + j];
-  }
-}
-
-QDEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-  hi = *reinterpret_cast<const uint16_t *>(&h);
-  lo = *reinterpret_cast<const uint16_t *>(&l);
-}
-
-// Projection reduction: out[m][j] = sum over splits (in order) of partial[sp][m][j];
-// then s*out split into bf16 hi/lo, written as hl [M, 2r] (hi in columns 0..r-1,
-// lo in r..2r-1) and/or hlT [2r, ldT].  Thread index runs over (j, m) with m fastest.
-__global__ void __launch_bounds__(256) proj_reduce_kernel(const float *__restrict__ partial, int splits,
-                                                          int M, int nn, int r, float s,
-                                                          float *__restrict__ out,
-                                                          uint16_t *__restrict__ hl,
-                                                          uint16_t *__restrict__ hlT, int ldT) {
-  const int64_t total = static_cast<int64_t>(M) * r;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int j = static_cast<int>(i / M);
-    const int m = static_cast<int>(i - static_cast<int64_t>(j) * M);
-    float v = 0.f;
-    for (int sp = 0; sp < splits; ++sp) v += partial[(static_cast<int64_t>(sp) * M + m) * nn + j];
-    if (out) out[static_cast<int64_t>(m) * r + j] = v;
-    uint16_t h, l;
-    split_hilo(s * v, h, l);
-    if (hl) {
-      hl[static_cast<int64_t>(m) * 2 * r + j] = h;
-      hl[static_cast<int64_t>(m) * 2 * r + r + j] = l;
-    }
-    if (hlT) {
-      hlT[static_cast<int64_t>(j) * ldT + m] = h;
-      hlT[static_cast<int64_t>(r + j) * ldT + m] = l;
-    }
   }
 }
 
@@ -227,27 +245,6 @@ __global__ void __launch_bounds__(256) hilo_t_kernel(const float *__restrict__ v
     split_hilo(s * v[static_cast<int64_t>(m) * r + j], h, l);
     hlT[static_cast<int64_t>(j) * ldT + m] = h;
     hlT[static_cast<int64_t>(r + j) * ldT + m] = l;
-  }
-}
-
-// Gradient reduction: g[c][j] = sum over splits of (partial[sp][c][j] + partial[sp][c][r+j])
-// (hi and lo halves).  layout 0 writes out[c][j] (dA [K, r]); layout 1 out[j][c] (dB [r, N]).
-__global__ void __launch_bounds__(256) grad_reduce_hilo_kernel(const float *__restrict__ partial,
-                                                               int splits, int C, int r, int layout,
-                                                               float *__restrict__ out) {
-  const int64_t total = static_cast<int64_t>(C) * r;
-  const int nn = 2 * r;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int64_t c, j;
-    if (layout == 0) { c = i / r; j = i - c * r; }
-    else { j = i / C; c = i - j * C; }
-    float v = 0.f;
-    for (int sp = 0; sp < splits; ++sp) {
-      const float *pp = partial + (static_cast<int64_t>(sp) * C + c) * nn;
-      v += pp[j] + pp[r + j];
-    }
-    out[i] = v;
   }
 }
 

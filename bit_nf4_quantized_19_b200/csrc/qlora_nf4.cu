@@ -69,7 +69,11 @@ qlora_status device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if (cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes) !=
+    if (cudaFuncSetAttribute(lora_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(lora_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes) !=
             cudaSuccess ||
         cudaFuncSetAttribute(qlora_xa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              xa_smem_bytes(64) > xa_smem_bytes(128) ? xa_smem_bytes(64) : xa_smem_bytes(128)) !=
@@ -182,10 +186,11 @@ struct Workspace {
 };
 
 // ---- launch geometry of the rank-r contractions (lora_mma_kernel)
+constexpr int kLmMaxSplits = 8;
+
 struct LmGeom {
   int nn, row_tiles, stages_total, sps, splits, num_stages;
   uint32_t tmem_cols;
-  size_t partial_bytes;
 };
 
 LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
@@ -195,36 +200,28 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   g.stages_total = static_cast<int>((contraction + 63) / 64);
   int want = (2 * sms + g.row_tiles - 1) / g.row_tiles;
   if (want < 1) want = 1;
+  if (want > kLmMaxSplits) want = kLmMaxSplits;     // the splits of a tile form one cluster
   if (want > g.stages_total) want = g.stages_total;
   g.sps = (g.stages_total + want - 1) / want;
   g.splits = (g.stages_total + g.sps - 1) / g.sps;
   int st = (110 * 1024) / (kLmABytes + nn * 128);
+  // the operand ring also holds the fp32 partial tile after the main loop
+  const int st_min = (kLmRows * nn * 4 + kLmABytes + nn * 128 - 1) / (kLmABytes + nn * 128);
+  if (st < st_min) st = st_min;
   g.num_stages = st < 2 ? 2 : (st > 8 ? 8 : st);
   uint32_t tc = 32;
   while (tc < static_cast<uint32_t>(nn)) tc <<= 1;
   g.tmem_cols = tc;
-  g.partial_bytes = static_cast<size_t>(g.splits) * static_cast<size_t>(rows) * nn * 4;
   return g;
 }
 
 int nn_proj(int r) { return (r + 15) / 16 * 16; }
 int64_t pad8(int64_t m) { return (m + 7) / 8 * 8; }
 
-size_t partial_max(int64_t M, int64_t N, int64_t K, int r, int sms) {
-  size_t a = lm_geom(M, K, nn_proj(r), sms).partial_bytes;
-  size_t b = lm_geom(M, N, nn_proj(r), sms).partial_bytes;
-  size_t c = lm_geom(K, M, 2 * r, sms).partial_bytes;
-  size_t d = lm_geom(N, M, 2 * r, sms).partial_bytes;
-  size_t x = a > b ? a : b;
-  size_t y = c > d ? c : d;
-  return x > y ? x : y;
-}
-
 size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
   b += align256(static_cast<size_t>(N) * (K / 64) * 4);        // expanded block constants
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T
-  b += align256(partial_max(M, N, K, r, sms));                 // split partials
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*XA hi/lo
   b += align256(static_cast<size_t>(M) * r * 4);               // XA when XA_out is NULL
   return b + 256;
@@ -234,7 +231,6 @@ size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
   b += align256(static_cast<size_t>(N) * (K / 64) * 4);
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T (XA recompute)
-  b += align256(partial_max(M, N, K, r, sms));
   b += align256(static_cast<size_t>(M) * r * 4);               // G
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*G hi/lo
   b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*G hi/lo transposed
@@ -274,12 +270,14 @@ int grid_for(int64_t total, int sms) {
   return g < 1 ? 1 : static_cast<int>(g);
 }
 
-// D[rows, nn] partials = act (K-major rows x c, or MN-major c x rows) * q^T, over splits.
+// D[rows, nn] = act (K-major rows x c, or MN-major c x rows) * q^T, split over the
+// contraction inside clusters of g.splits CTAs that reduce in rank order; the final
+// outputs are written by the kernel (projection or gradient form, see LoraMmaParams).
 template <bool A_MN>
 qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_cols,
                              const uint16_t *qop, int64_t q_rows, int64_t q_cols, int64_t q_pitch,
-                             int64_t rows, int64_t contraction, int nn, float *partial, int sms,
-                             cudaStream_t st, LmGeom *geom_out) {
+                             int64_t rows, int64_t contraction, int nn, LoraMmaParams p, int sms,
+                             cudaStream_t st) {
   const LmGeom g = lm_geom(rows, contraction, nn, sms);
   CUtensorMap tm_act, tm_q;
   // act is [act_rows (tokens), act_cols (features)] row-major bf16
@@ -289,46 +287,50 @@ qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_
   if (!make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qop, q_cols, q_rows, q_pitch * 2, 64,
                    static_cast<uint32_t>(nn), CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
-  LoraMmaParams p{};
   p.rows = static_cast<int>(rows);
   p.nn = nn;
   p.stages_total = g.stages_total;
   p.stages_per_split = g.sps;
   p.num_stages = g.num_stages;
   p.tmem_cols = g.tmem_cols;
-  p.partial = partial;
+  p.splits = g.splits;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
   const int smem = lora_mma_smem_bytes(nn, g.num_stages);
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[A_MN ? 1 : 0]) {
-    if (cudaFuncSetAttribute(lora_mma_kernel<A_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    attr_set[A_MN ? 1 : 0] = true;
-  }
-  dim3 grid(static_cast<unsigned>(g.row_tiles), static_cast<unsigned>(g.splits));
+  if (smem > 200 * 1024) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(g.row_tiles), static_cast<unsigned>(g.splits), 1);
+  cfg.blockDim = dim3(kLmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(g.splits);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   LaunchTimer lt(A_MN ? QLORA_K_GRAD : QLORA_K_PROJECT, st);
-  lora_mma_kernel<A_MN><<<grid, kLmThreads, smem, st>>>(tm_act, tm_q, p);
-  if (geom_out) *geom_out = g;
-  return cuda_status(cudaGetLastError());
+  return cuda_status(cudaLaunchKernelEx(&cfg, lora_mma_kernel<A_MN>, tm_act, tm_q, p));
 }
 
 // XA = X A (or G = dY B^T): fp32 [M, r] plus hi/lo of s*result in [M, 2r] and/or [2r, pad8(M)].
 qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const uint16_t *qT,
-                               int r, float s, float *out, uint16_t *hl, uint16_t *hlT,
-                               float *partial, int sms, cudaStream_t st) {
-  LmGeom g;
-  qlora_status e = launch_lora_mma<false>(act, M, C, qT, r, C, C, M, C, nn_proj(r), partial, sms, st, &g);
-  if (e != QLORA_OK) return e;
-  LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
-  proj_reduce_kernel<<<grid_for(M * r, sms), 256, 0, st>>>(partial, g.splits, static_cast<int>(M), g.nn,
-                                                           r, s, out, hl, hlT, static_cast<int>(pad8(M)));
-  return cuda_status(cudaGetLastError());
+                               int r, float s, float *out, uint16_t *hl, uint16_t *hlT, int sms,
+                               cudaStream_t st) {
+  LoraMmaParams p{};
+  p.grad = 0;
+  p.r = r;
+  p.s = s;
+  p.out = out;
+  p.hl = hl;
+  p.hlT = hlT;
+  p.ldT = static_cast<int>(pad8(M));
+  return launch_lora_mma<false>(act, M, C, qT, r, C, C, M, C, nn_proj(r), p, sms, st);
 }
 
 qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *hlT, int sms,
                            cudaStream_t st) {
-  LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
+  LaunchTimer lt(QLORA_K_EXPAND, st);
   hilo_t_kernel<<<grid_for(M * r, sms), 256, 0, st>>>(v, static_cast<int>(M), r, s, hlT,
                                                        static_cast<int>(pad8(M)));
   return cuda_status(cudaGetLastError());
@@ -336,15 +338,13 @@ qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *
 
 // g = act^T * (hi + lo) over tokens: act [M, C] bf16, hlT [2r, pad8(M)]; out dA [C, r] or dB [r, C].
 qlora_status launch_grad(const uint16_t *act, int64_t M, int64_t C, const uint16_t *hlT, int r,
-                         int layout, float *out, float *partial, int sms, cudaStream_t st) {
-  LmGeom g;
-  qlora_status e = launch_lora_mma<true>(act, M, C, hlT, 2 * r, M, pad8(M), C, M, 2 * r, partial, sms,
-                                         st, &g);
-  if (e != QLORA_OK) return e;
-  LaunchTimer lt(QLORA_K_GRAD_REDUCE, st);
-  grad_reduce_hilo_kernel<<<grid_for(C * r, sms), 256, 0, st>>>(partial, g.splits, static_cast<int>(C), r,
-                                                                layout, out);
-  return cuda_status(cudaGetLastError());
+                         int layout, float *out, int sms, cudaStream_t st) {
+  LoraMmaParams p{};
+  p.grad = 1;
+  p.r = r;
+  p.out = out;
+  p.layout = layout;
+  return launch_lora_mma<true>(act, M, C, hlT, 2 * r, M, pad8(M), C, M, 2 * r, p, sms, st);
 }
 
 qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT, int sms, cudaStream_t st) {
@@ -656,13 +656,12 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
-  float *part = static_cast<float *>(ws.take(partial_max(M, N, K, r, d->sms)));
   uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  if (!S || !AT || !part || !hl || !xa) return QLORA_ERR_WORKSPACE;
+  if (!S || !AT || !hl || !xa) return QLORA_ERR_WORKSPACE;
   // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps
   if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, part, d->sms, stream)) != QLORA_OK)
+  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream)) != QLORA_OK)
     return st;
   if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
   return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, d->sms, stream);
@@ -689,30 +688,29 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
   const size_t hlT_bytes = static_cast<size_t>(2 * r) * pad8(M) * 2;
   float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
-  float *part = static_cast<float *>(ws.take(partial_max(M, N, K, r, d->sms)));
   float *G = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   uint16_t *ghl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   uint16_t *ghlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  if (!S || !AT || !part || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
+  if (!S || !AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
   // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from X and A)
   if (XA) {
     if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
   } else {
     if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-    if ((st = launch_projection(X, M, K, AT, r, s, xa_ws, nullptr, xahlT, part, d->sms, stream)) != QLORA_OK)
+    if ((st = launch_projection(X, M, K, AT, r, s, xa_ws, nullptr, xahlT, d->sms, stream)) != QLORA_OK)
       return st;
   }
   // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA)
-  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, part, d->sms, stream)) != QLORA_OK) return st;
+  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream)) != QLORA_OK) return st;
   if (dX) {
     if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
     if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, d->sms, stream)) != QLORA_OK) return st;
   }
   // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
-  if ((st = launch_grad(X, M, K, ghlT, r, 0, dA, part, d->sms, stream)) != QLORA_OK) return st;
-  return launch_grad(dY, M, N, xahlT, r, 1, dB, part, d->sms, stream);
+  if ((st = launch_grad(X, M, K, ghlT, r, 0, dA, d->sms, stream)) != QLORA_OK) return st;
+  return launch_grad(dY, M, N, xahlT, r, 1, dB, d->sms, stream);
 }
 
 qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags) {

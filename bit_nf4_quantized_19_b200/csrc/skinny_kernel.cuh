@@ -59,25 +59,6 @@ struct SkinnyParams {
   float levels[16];
 };
 
-QDEV uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-QDEV void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Shared-memory address of the same variable in CTA `rank` of the cluster.
-QDEV uint32_t map_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-QDEV float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
 // Two transposed 8x8 bf16 tiles: lanes 0-7 address the rows of the first, 8-15
 // of the second; lane 4g+c receives rows 2c, 2c+1 of column g of each.
 QDEV void ldmatrix_x2_trans(uint32_t addr, uint32_t &b0, uint32_t &b1) {

@@ -218,12 +218,14 @@ uint32_t qlora_set_wait_limit_us(uint32_t limit_us);
 typedef enum {
   QLORA_K_QUANTIZE = 0,     /* nf4 quantize + double quant          */
   QLORA_K_DEQUANT = 1,      /* standalone dequant                   */
-  QLORA_K_EXPAND = 2,       /* block-constant expansion for a GEMM  */
+  QLORA_K_EXPAND = 2,       /* operand preparation: block-constant  */
+                            /* expansion, A^T, hi/lo of a saved XA  */
   QLORA_K_PROJECT = 3,      /* XA = X A or G = dY B^T (+ hi/lo)     */
   QLORA_K_GEMM_FWD = 4,     /* fused dequant GEMM, forward          */
   QLORA_K_GEMM_DX = 5,      /* fused dequant GEMM, dX               */
-  QLORA_K_GRAD = 6,         /* adapter-gradient partial sums        */
-  QLORA_K_GRAD_REDUCE = 7,  /* adapter-gradient reduction           */
+  QLORA_K_GRAD = 6,         /* adapter gradients dA, dB             */
+  QLORA_K_GRAD_REDUCE = 7,  /* unused: the split sums now happen    */
+                            /* inside the QLORA_K_GRAD launches     */
   QLORA_K_SKINNY = 8        /* few-token forward                    */
 } qlora_kernel_kind;
 
