@@ -43,7 +43,24 @@ struct DeviceInfo {
   int sms = 0;
   int major = 0;
   bool gemm_attr_set = false;
+  // A second stream of the library's own, for work that only depends on the weight
+  // (the block-constant expansion) to run beside the rank-r projection.  fork_mu
+  // keeps each fork / join pair of event records and waits together.
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  std::mutex fork_mu;
 };
+// Joins the side stream back into the caller's stream when a forked call leaves
+// early on an error, so no side-stream work outlives the call's ordering.
+struct ForkGuard {
+  DeviceInfo *d;
+  cudaStream_t st;
+  bool pending = false;
+  ~ForkGuard() {
+    if (pending) cudaStreamWaitEvent(st, d->ev_join, 0);
+  }
+};
+
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -61,6 +78,12 @@ qlora_status device_info(DeviceInfo **out) {
       return QLORA_ERR_CUDA;
     d.sms = sms;
     d.major = major;
+    if (cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.ev_join, cudaEventDisableTiming) != cudaSuccess) {
+      d.sms = 0;
+      return QLORA_ERR_CUDA;
+    }
   }
   if (d.major != 10) return QLORA_ERR_NO_DEVICE;
   if (!d.gemm_attr_set) {
@@ -660,10 +683,23 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
   float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   if (!S || !AT || !hl || !xa) return QLORA_ERR_WORKSPACE;
   // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps
-  if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream)) != QLORA_OK)
-    return st;
-  if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
+  {
+    // the block constants depend only on the weight: expand them on the side stream
+    // while X*A runs here, and join before the GEMM
+    std::lock_guard<std::mutex> lk(d->fork_mu);
+    if (cudaEventRecord(d->ev_fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    ForkGuard fg{d, stream};
+    if ((st = launch_expand_scales(Wq, S, d->side, d->sms)) != QLORA_OK) return st;
+    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess) return QLORA_ERR_CUDA;
+    fg.pending = true;
+    if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+    if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream)) != QLORA_OK)
+      return st;
+    fg.pending = false;
+    if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
   return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, d->sms, stream);
 }
 
@@ -694,6 +730,19 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
   uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   if (!S || !AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
+  std::unique_lock<std::mutex> lk(d->fork_mu, std::defer_lock);
+  ForkGuard fg{d, stream};
+  if (dX) {
+    // the block constants depend only on the weight: expand them on the side stream
+    // while the rank-r products below run here, and join before the dX GEMM
+    lk.lock();
+    if (cudaEventRecord(d->ev_fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    if ((st = launch_expand_scales(Wq, S, d->side, d->sms)) != QLORA_OK) return st;
+    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess) return QLORA_ERR_CUDA;
+    fg.pending = true;
+  }
   // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from X and A)
   if (XA) {
     if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
@@ -705,7 +754,9 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
   // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA)
   if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream)) != QLORA_OK) return st;
   if (dX) {
-    if ((st = launch_expand_scales(Wq, S, stream, d->sms)) != QLORA_OK) return st;
+    fg.pending = false;
+    if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
+    lk.unlock();
     if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, d->sms, stream)) != QLORA_OK) return st;
   }
   // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]

@@ -148,3 +148,39 @@ def test_gemm_dequant_bit_exact_one_hot(q, N, K):
     torch.cuda.synchronize()
     assert np.array_equal(H.dev_to_bits(Y), ref.T)
     assert np.array_equal(H.dev_to_bits(dX), ref)
+
+
+def test_fwd_bwd_capture_in_cuda_graph(q):
+    """The forward and backward (which fork the block-constant expansion onto the
+    library's side stream and join it back) capture into one CUDA graph; replays
+    give bit-identical results to eager calls."""
+    import torch
+    p = linear_problem(64, 384, 512, 16, 32.0, 0.02, seed=3)
+    X, A, B, dY = (H.bits_to_dev(v) for v in (p.X, p.A, p.B, p.dY))
+    Wq = q.nf4_quantize(H.bits_to_dev(p.W))
+    ws = q.make_workspace(p.M, p.N, p.K, p.r, X.device)
+    Y = torch.empty(p.M, p.N, dtype=torch.bfloat16, device="cuda")
+    XA = torch.empty(p.M, p.r, dtype=torch.float32, device="cuda")
+    dX = torch.empty(p.M, p.K, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(p.K, p.r, dtype=torch.float32, device="cuda")
+    dB = torch.empty(p.r, p.N, dtype=torch.float32, device="cuda")
+
+    def step():
+        q.linear_fwd(X, Wq, A, B, p.s, workspace=ws, Y=Y, XA=XA)
+        q.linear_bwd(dY, X, XA, Wq, A, B, p.s, workspace=ws, dX=dX, dA=dA, dB=dB)
+
+    step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (Y, XA, dX, dA, dB)]
+    for t in (Y, XA, dX, dA, dB):
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert q.device_status() == (0, 0)
+    for got, want in zip((Y, XA, dX, dA, dB), ref):
+        assert torch.equal(got.view(torch.int16) if got.dtype == torch.bfloat16 else got.view(torch.int32),
+                           want.view(torch.int16) if want.dtype == torch.bfloat16 else want.view(torch.int32))
