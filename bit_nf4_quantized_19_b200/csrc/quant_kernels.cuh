@@ -24,10 +24,10 @@ struct Levels {
   float v[16];
 };
 
-// Persistent CTAs (three per SM), each looping over groups of 256 blocks (16384
-// values); 256 threads; 8 threads per block, each owning 8 consecutive values (one
-// 16-byte load), 32 blocks per pass, 8 passes.  All eight 16-byte loads of a group
-// are issued before any arithmetic.
+// Persistent CTAs (one per SM), each looping over groups of 256 blocks (16384
+// values); 512 threads; 8 threads per block, each owning 8 consecutive values (one
+// 16-byte piece), 64 blocks per pass, 4 passes; the groups arrive through a ring of
+// bulk copies (see the kernel).
 //   absmax: max |w| within the thread, then an xor-shuffle over the 8 lanes;
 //   xn:     RN32(w / a_b).  For 2^-64 <= a_b <= 2^64 (every realistic block) the
 //           division is Markstein's FMA correction of w * RN32(1/a_b), where
@@ -75,16 +75,17 @@ QDEV uint32_t bmax2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// The eight 16-byte loads of one thread for one group (pass p: block 32 p + bl,
-// values 8 sub .. 8 sub + 7); WHOLE = the group lies entirely inside the tensor.
-template <bool WHOLE>
-QDEV void quant_load(const uint16_t *__restrict__ W, int64_t n, int64_t gbase, int bl, int sub, uint4 (&v)[8]) {
-  const uint16_t *base = W + gbase + bl * kBlock + sub * 8;
+// The NP 16-byte loads of one thread for one group straight from global memory
+// (pass p: block (256/NP) p + bl, values 8 sub .. 8 sub + 7), with bounds checks:
+// the path of the one group that may end inside the tensor.
+template <int NP>
+QDEV void quant_load_tail(const uint16_t *__restrict__ W, int64_t n, int64_t gbase, int bl, int sub, uint4 (&v)[NP]) {
+  constexpr int BPP = kGroup / NP;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int64_t e = gbase + static_cast<int64_t>(p * 32 + bl) * kBlock + sub * 8;
-    if (WHOLE || e + 8 <= n) {
-      v[p] = ld_global_nc_v4(base + p * 32 * kBlock);
+  for (int p = 0; p < NP; ++p) {
+    const int64_t e = gbase + static_cast<int64_t>(p * BPP + bl) * kBlock + sub * 8;
+    if (e + 8 <= n) {
+      v[p] = ld_global_nc_v4(W + e);
     } else {
       uint32_t t[4] = {0, 0, 0, 0};
       for (int j = 0; j < 8; ++j)
@@ -97,13 +98,14 @@ QDEV void quant_load(const uint16_t *__restrict__ W, int64_t n, int64_t gbase, i
 // Codes of one group.  The eight block absmaxes come first, on the packed bf16
 // words (|w| is w with the sign bits cleared; NaN propagates), two passes per
 // shuffle; one warp vote then picks the path for the whole group.
-template <bool WHOLE>
-QDEV void quant_compute(const uint4 (&v)[8], int64_t n, int64_t gbase, int bl, int sub, const float *rcp,
+template <bool WHOLE, int NP>
+QDEV void quant_compute(const uint4 (&v)[NP], int64_t n, int64_t gbase, int bl, int sub, const float *rcp,
                         const uint8_t *bins_bytes, uint32_t lane8, uint8_t *__restrict__ codes,
                         float *amax, bool &nonfinite) {
-  float am[8];
+  constexpr int BPP = kGroup / NP;
+  float am[NP];
 #pragma unroll
-  for (int p = 0; p < 8; p += 2) {
+  for (int p = 0; p < NP; p += 2) {
     uint32_t m0 = bmax2(bmax2(v[p].x & 0x7FFF7FFFu, v[p].y & 0x7FFF7FFFu), bmax2(v[p].z & 0x7FFF7FFFu, v[p].w & 0x7FFF7FFFu));
     uint32_t m1 = bmax2(bmax2(v[p + 1].x & 0x7FFF7FFFu, v[p + 1].y & 0x7FFF7FFFu),
                         bmax2(v[p + 1].z & 0x7FFF7FFFu, v[p + 1].w & 0x7FFF7FFFu));
@@ -117,12 +119,12 @@ QDEV void quant_compute(const uint4 (&v)[8], int64_t n, int64_t gbase, int bl, i
   }
   bool fast = true;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) fast = fast && (am[p] >= 0x1p-64f) && (am[p] <= 0x1p64f);
+  for (int p = 0; p < NP; ++p) fast = fast && (am[p] >= 0x1p-64f) && (am[p] <= 0x1p64f);
   const bool group_fast = __all_sync(0xffffffffu, fast);
   uint8_t *cbase = codes + ((gbase + bl * kBlock + sub * 8) >> 1);
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int64_t e = gbase + static_cast<int64_t>(p * 32 + bl) * kBlock + sub * 8;
+  for (int p = 0; p < NP; ++p) {
+    const int64_t e = gbase + static_cast<int64_t>(p * BPP + bl) * kBlock + sub * 8;
     const uint32_t wd[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
     float w[8];
 #pragma unroll
@@ -168,7 +170,7 @@ QDEV void quant_compute(const uint4 (&v)[8], int64_t n, int64_t gbase, int bl, i
       }
     }
     if (WHOLE || e + 8 <= n) {
-      *reinterpret_cast<uint32_t *>(cbase + p * 32 * kBlock / 2) = word;
+      *reinterpret_cast<uint32_t *>(cbase + p * BPP * kBlock / 2) = word;
     } else if (e < n) {
       const int valid = static_cast<int>(n - e);           // 1..7
       const uint32_t keep = (1u << (4 * valid)) - 1u;      // zero the nibbles past n
@@ -176,67 +178,112 @@ QDEV void quant_compute(const uint4 (&v)[8], int64_t n, int64_t gbase, int bl, i
       const int nbytes = (valid + 1) >> 1;
       for (int j = 0; j < nbytes; ++j) codes[(e >> 1) + j] = static_cast<uint8_t>(word >> (8 * j));
     }
-    if (sub == 0) amax[p * 32 + bl] = a_b;
+    if (sub == 0) amax[p * BPP + bl] = a_b;
   }
 }
 
-constexpr int kQuantCtasPerSm = 3;
-constexpr int kQuantSmemBytes = kQuantBins256 * 32 * 8 + (128 + 256 + 8) * 4;
+// One persistent CTA of 512 threads per SM.  The groups this CTA owns stream
+// through a ring of kQuantStages 32 KB buffers, each filled by one bulk copy on its
+// own mbarrier (kept kQuantStages groups ahead), so the SM always has about
+// 128 KB of loads in flight whatever the compute is doing; the compute reads its
+// 16-byte pieces from shared memory (consecutive threads, consecutive pieces).  The
+// one group that may end inside the tensor takes bounds-checked global loads.
+constexpr int kQuantThreads = 512;
+constexpr int kQuantStages = 4;
+constexpr int kQuantPasses = kGroupElems / (kQuantThreads * 8);   // 4
+constexpr int kQuantStageBytes = kGroupElems * 2;                 // 32 KB
+constexpr int kQuantSmemBytes = kQuantStages * kQuantStageBytes + kQuantBins256 * 32 * 8 +
+                                (128 + kGroup + 16) * 4 + kQuantStages * 8 + 16;
 
-__global__ void __launch_bounds__(256, kQuantCtasPerSm) nf4_quantize_kernel(
+__global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(
     const uint16_t *__restrict__ W, int64_t n, uint8_t *__restrict__ codes,
-    uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab) {
-  extern __shared__ __align__(16) uint8_t qsm[];
-  uint2 *bins = reinterpret_cast<uint2 *>(qsm);                          // [256 entries][32 lanes]: (t bits, c)
-  float *rcp = reinterpret_cast<float *>(qsm + kQuantBins256 * 32 * 8);  // [128]
-  float *amax = rcp + 128;                                               // [256]
-  float *wmax = amax + kGroup;                                           // [8]
+    uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab,
+    uint64_t limit_ns) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  uint8_t *ring = qsm;                                                             // [stages][32 KB]
+  uint8_t *bins_bytes = qsm + kQuantStages * kQuantStageBytes;
+  uint2 *bins = reinterpret_cast<uint2 *>(bins_bytes);                             // [256 entries][32 lanes]
+  float *rcp = reinterpret_cast<float *>(bins_bytes + kQuantBins256 * 32 * 8);     // [128]
+  float *amax = rcp + 128;                                                         // [256]
+  float *wmax = amax + kGroup;                                                     // [16]
+  uint64_t *full = reinterpret_cast<uint64_t *>(wmax + 16);                        // [stages]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(full + kQuantStages);
   const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < kQuantBins256 * 32; i += 256) {
+  const int64_t ngroups = (n + kGroupElems - 1) / kGroupElems;
+  const int64_t nblocks = (n + kBlock - 1) / kBlock;
+  const int64_t G = gridDim.x;
+  auto whole = [&](int64_t g) { return (g + 1) * kGroupElems <= n; };
+
+  for (int i = tid; i < kQuantBins256 * 32; i += kQuantThreads) {
     const QuantBin e = tab.bins[i >> 5];
     bins[i] = make_uint2(__float_as_uint(e.t), static_cast<uint32_t>(e.c));
   }
   if (tid < 128) rcp[tid] = tab.rcp[tid];
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int k = 0; k < kQuantStages; ++k) mbar_init(&full[k], 1);
+    fence_mbar_init();
+    for (int k = 0; k < kQuantStages; ++k) {
+      const int64_t g = blockIdx.x + k * G;
+      if (g < ngroups && whole(g)) {
+        mbar_arrive_expect_tx(&full[k], kQuantStageBytes);
+        bulk_load(ring + k * kQuantStageBytes, W + g * kGroupElems, kQuantStageBytes, &full[k]);
+      }
+    }
+  }
+  const Waiter waiter{abort_flag, limit_ns};
   const uint32_t lane8 = 8u * static_cast<uint32_t>(lane);
-  const uint8_t *bins_bytes = qsm;
   const int sub = tid & 7;
-  const int bl = tid >> 3;
-  const int64_t ngroups = (n + kGroupElems - 1) / kGroupElems;
-  const int64_t nblocks = (n + kBlock - 1) / kBlock;
+  const int bl = tid >> 3;                     // block within a pass (0..63)
   bool nonfinite = false;
 
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+  int it = 0;
+  for (int64_t g = blockIdx.x; g < ngroups; g += G, ++it) {
+    const int s = it % kQuantStages;
+    const uint32_t ph = static_cast<uint32_t>(it / kQuantStages) & 1u;
     const int64_t gbase = g * kGroupElems;
-    uint4 v[8];
-    if (gbase + kGroupElems <= n) {
-      quant_load<true>(W, n, gbase, bl, sub, v);
-      __syncthreads();   // tables filled; the previous group's amax and wmax consumed
-      quant_compute<true>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
+    __syncthreads();   // tables and barriers ready; the previous group's amax and wmax consumed
+    uint4 v[kQuantPasses];
+    if (whole(g)) {
+      if (!__syncthreads_and(wait_bar(&full[s], ph, waiter))) break;
+      const uint32_t src = smem_u32(ring + s * kQuantStageBytes) + static_cast<uint32_t>((bl * kBlock + sub * 8) * 2);
+#pragma unroll
+      for (int p = 0; p < kQuantPasses; ++p)
+        v[p] = ld_shared_v4(src + static_cast<uint32_t>(p * (kGroup / kQuantPasses) * kBlock * 2));
+      quant_compute<true, kQuantPasses>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
     } else {
-      quant_load<false>(W, n, gbase, bl, sub, v);
-      __syncthreads();
-      quant_compute<false>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
+      quant_load_tail<kQuantPasses>(W, n, gbase, bl, sub, v);
+      quant_compute<false, kQuantPasses>(v, n, gbase, bl, sub, rcp, bins_bytes, lane8, codes, amax, nonfinite);
     }
-    __syncthreads();
+    __syncthreads();   // stage s consumed, the group's block absmaxes complete
+    if (tid == 0) {
+      const int64_t gn = g + kQuantStages * G;
+      if (gn < ngroups && whole(gn)) {
+        mbar_arrive_expect_tx(&full[s], kQuantStageBytes);
+        bulk_load(ring + s * kQuantStageBytes, W + gn * kGroupElems, kQuantStageBytes, &full[s]);
+      }
+    }
 
-    // second level: one constant per group
+    // second level: one constant per group (threads 0..255, one block each)
     const int64_t b = g * kGroup + tid;
-    const float a = (b < nblocks) ? amax[tid] : 0.f;
+    const float a = (tid < kGroup && b < nblocks) ? amax[tid] : 0.f;
     float m = a;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((tid & 31) == 0) wmax[tid >> 5] = m;
+    if (lane == 0 && tid < kGroup) wmax[tid >> 5] = m;
     __syncthreads();
-    float c = wmax[0];
+    if (tid < kGroup) {
+      float c = wmax[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) c = fmaxf(c, wmax[i]);
-    const float st = (c > 0.f) ? __fdiv_rn(c, 255.0f) : 0.f;
-    if (b < nblocks) {
-      int q = 0;
-      if (c > 0.f) q = min(255, __float2int_rn(__fdiv_rn(a, st)));
-      q8[b] = static_cast<uint8_t>(q);
+      for (int i = 1; i < kGroup / 32; ++i) c = fmaxf(c, wmax[i]);
+      const float st = (c > 0.f) ? __fdiv_rn(c, 255.0f) : 0.f;
+      if (b < nblocks) {
+        int q = 0;
+        if (c > 0.f) q = min(255, __float2int_rn(__fdiv_rn(a, st)));
+        q8[b] = static_cast<uint8_t>(q);
+      }
+      if (tid == 0) step[g] = st;
     }
-    if (tid == 0) step[g] = st;
   }
   if (nonfinite && sub == 0) atomicOr(&g_device_status, kStatNonFinite);
 }
