@@ -28,6 +28,15 @@
 //                 thread, decoded through a 16-entry table held in registers),
 //                 then the LoRA weight tiles.
 // Every wait is bounded (see Waiter); a wait that runs out aborts the block.
+//
+// Last-wave split: with T tiles on G persistent CTAs, T mod G tiles are left for a
+// last round in which most SMs would idle.  When at most G/2 remain, each of them
+// is split along the contraction into two halves taken by CTAs 2i and 2i+1: the
+// first half writes its fp32 partial tile to scratch and publishes it under a
+// per-launch epoch (release); the second half runs the rest of the contraction and
+// the LoRA steps, waits for the epoch (acquire, bounded), and adds the partial in
+// its epilogue.  The first half never waits, and the grid has at most one CTA per
+// SM, so the wait always ends.
 #pragma once
 #include "common.cuh"
 
@@ -74,8 +83,49 @@ struct GemmParams {
   const uint16_t *lora_w;  // fwd: B [r, N];  dX: A [K, r]
   uint16_t *out;     // Y [M, N] or dX [M, K]
   uint64_t limit_ns;
+  int split_base;    // first tile of the split last round (a multiple of the grid size)
+  int split_count;   // tiles split into two contraction halves (0: no split)
+  int kb_mid;        // first main stage of the second half
+  float *scratch;    // [split_count][128][256] fp32 partial tiles of the first halves
+  unsigned long long *flags;   // [split_count]: epoch once the partial tile is complete
+  unsigned long long epoch;    // unique per launch
   float levels[16];
 };
+
+// The work items of this CTA: whole tiles blockIdx.x + i*G below split_base, then
+// (when a last round is split) one half of tile split_base + blockIdx.x/2: part 1
+// = main stages [0, kb_mid), part 2 = [kb_mid, kb_main) plus the LoRA stages.
+struct GemmItem {
+  int tile, kb0, kb1, part;
+  bool lora;
+};
+
+QDEV bool gemm_item(const GemmParams &p, int num_tiles, int it, GemmItem &w) {
+  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  const int whole_end = p.split_count ? p.split_base : num_tiles;
+  const int t = b + it * G;
+  if (t < whole_end) {
+    w.tile = t; w.kb0 = 0; w.kb1 = p.kb_main; w.part = 0; w.lora = true;
+    return true;
+  }
+  if (!p.split_count || it != whole_end / G || b >= 2 * p.split_count) return false;
+  w.tile = p.split_base + (b >> 1);
+  w.part = 1 + (b & 1);
+  w.kb0 = (w.part == 1) ? 0 : p.kb_mid;
+  w.kb1 = (w.part == 1) ? p.kb_mid : p.kb_main;
+  w.lora = (w.part == 2);
+  return true;
+}
+
+QDEV unsigned long long ld_acquire_u64(const unsigned long long *a) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+  return v;
+}
+QDEV void st_release_u64(unsigned long long *a, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(v) : "memory");
+}
+QDEV void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -138,7 +188,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const Waiter wt{abort_flag, p.limit_ns};
 
   const int num_tiles = p.num_m_tiles * p.num_w_tiles;
-  const int nkb = p.kb_main + p.kb_lora;
 
   if (warp == 0) {
     // ------------------------------------------------------------ activation producer
@@ -147,15 +196,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t bph = 0;
       uint32_t armedB = 0, lastB = 0;          // bit s: armed at least once / parity of last arming
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int m0 = (tile / p.num_w_tiles) * kBN;
-        for (int kb = 0; kb < nkb; ++kb) {
+      GemmItem w;
+      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
+        const int m0 = (w.tile / p.num_w_tiles) * kBN;
+        const int nmain = w.kb1 - w.kb0, nst = nmain + (w.lora ? p.kb_lora : 0);
+        for (int j = 0; j < nst; ++j) {
           if (!wait_bar(&empty_A[bs], bph ^ 1u, wt)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_B[bs], kBStageBytes);
-          if (kb < p.kb_main)
-            tma_load_2d(sB + bs * kBStageBytes, &tm_act, &full_B[bs], kb * kBK, m0);
+          if (j < nmain)
+            tma_load_2d(sB + bs * kBStageBytes, &tm_act, &full_B[bs], (w.kb0 + j) * kBK, m0);
           else
-            tma_load_2d(sB + bs * kBStageBytes, &tm_lora, &full_B[bs], (kb - p.kb_main) * kBK, m0);
+            tma_load_2d(sB + bs * kBStageBytes, &tm_lora, &full_B[bs], (j - nmain) * kBK, m0);
           armedB |= 1u << bs;
           lastB = (lastB & ~(1u << bs)) | (bph << bs);
           if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
@@ -174,9 +225,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t wph = 0;
       uint32_t armedW = 0, lastW = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int w0 = (tile % p.num_w_tiles) * kWT;
-        for (int kb = 0; kb < p.kb_main; ++kb) {
+      GemmItem w;
+      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
+        const int w0 = (w.tile % p.num_w_tiles) * kWT;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!wait_bar(&empty_W[ws], wph ^ 1u, wt)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_W[ws], kWStageBytes + kSStageBytes);
           if (MODE == kModeFwd) {
@@ -214,16 +266,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t ad_main0 = (MODE == kModeDx) ? sw128_desc(a0, 1024, 2048) : sw128_desc(a0, 16, 1024);
       const uint64_t ad_lora0 = (MODE == kModeFwd) ? sw128_desc(a0, 1024, 2048) : sw128_desc(a0, 16, 1024);
       const uint64_t bd0 = sw128_desc(b0, 16, 1024);
-      const int kb_main = p.kb_main, kb_lora = p.kb_lora;
+      const int kb_lora = p.kb_lora;
       const int lora_steps_total = (2 * p.r) / 16;
       int st = 0, acc = 0;
       uint32_t ph = 0, accph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      GemmItem w;
+      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
         if (!wait_bar(&tmem_empty[acc], accph ^ 1u, wt)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kb = 0; kb < kb_main; ++kb) {
+        for (int kb = 0; kb < w.kb1 - w.kb0; ++kb) {
           if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = ad_main0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
@@ -234,7 +287,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mma_commit(&empty_A[st]);
           if (++st == kStagesA) { st = 0; ph ^= 1u; }
         }
-        for (int ls = 0; ok && ls < kb_lora; ++ls) {
+        for (int ls = 0; ok && w.lora && ls < kb_lora; ++ls) {
           if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = ad_lora0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
@@ -261,13 +314,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = q * 32 + lane;      // weight-side row within the tile
     int acc = 0;
     uint32_t accph = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int m0 = (tile / p.num_w_tiles) * kBN;
-      const int w0 = (tile % p.num_w_tiles) * kWT;
+    GemmItem w;
+    for (int it = 0; gemm_item(p, num_tiles, it, w); ++it) {
+      const int m0 = (w.tile / p.num_w_tiles) * kBN;
+      const int w0 = (w.tile % p.num_w_tiles) * kWT;
       // warp-uniform decision: the TMEM loads below are .sync.aligned
       const bool got = __all_sync(0xffffffffu, wait_bar(&tmem_full[acc], accph, wt) ? 1 : 0);
       if (!got) break;
       tc_fence_after();
+      const int sidx = w.tile - p.split_base;                  // split tiles only
+      float *prow = (w.part != 0) ? p.scratch + (static_cast<int64_t>(sidx) * kWT + row) * kBN : nullptr;
+      if (w.part == 2) {
+        // the first half's partial tile: one thread waits for its epoch (bounded)
+        if (warp == 4 && lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_u64(p.flags + sidx) != p.epoch) {
+            if (*reinterpret_cast<volatile int *>(abort_flag) || globaltimer_ns() - t0 > p.limit_ns) {
+              *reinterpret_cast<volatile int *>(abort_flag) = 1;
+              atomicOr(&g_device_status, kStatTimeout);
+              break;
+            }
+          }
+        }
+        epilogue_bar();
+        __threadfence();
+      }
       uint16_t *outc = p.out + w0 + row;
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t v[32];
@@ -275,6 +346,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                static_cast<uint32_t>(acc * kBN + cc * 32),
                            v);
         tmem_wait_ld();
+        if (w.part == 1) {
+          float4 *d4 = reinterpret_cast<float4 *>(prow + cc * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          continue;
+        }
+        if (w.part == 2) {
+          const float4 *s4 = reinterpret_cast<const float4 *>(prow + cc * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 f = __ldcg(s4 + j);
+            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + f.x);
+            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + f.y);
+            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + f.z);
+            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + f.w);
+          }
+        }
         const int mb = m0 + cc * 32;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -284,6 +374,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             outc[static_cast<int64_t>(m) * p.n_out] = *reinterpret_cast<const uint16_t *>(&h);
           }
         }
+      }
+      if (w.part == 1) {
+        // publish the partial tile: every epilogue thread's stores, then one release
+        __threadfence();
+        epilogue_bar();
+        if (warp == 4 && lane == 0) st_release_u64(p.flags + sidx, p.epoch);
       }
       tc_fence_before();
       __syncwarp();
@@ -299,10 +395,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int i = 0; i < 16; ++i) L[i] = sL[i];
     uint32_t a_cnt = 0, w_cnt = 0;      // stages seen so far (all / main only)
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      const int w0 = (tile % p.num_w_tiles) * kWT;
-      for (int kb = 0; kb < nkb; ++kb, ++a_cnt) {
-        const bool main = kb < p.kb_main;
+    GemmItem w;
+    for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
+      const int w0 = (w.tile % p.num_w_tiles) * kWT;
+      const int nmain = w.kb1 - w.kb0, nst = nmain + (w.lora ? p.kb_lora : 0);
+      for (int j = 0; j < nst; ++j, ++a_cnt) {
+        const bool main = j < nmain;
         const uint32_t my_w = w_cnt;
         if (main) ++w_cnt;
         if ((a_cnt & 1u) != static_cast<uint32_t>(grp)) continue;
@@ -350,7 +448,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) mbar_arrive(&full_A[as]);
         } else {
           // LoRA weight-side stage: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
-          const int ls = kb - p.kb_main;
+          const int ls = j - nmain;
           if (!__all_sync(0xffffffffu, wait_bar(&empty_A[as], aph ^ 1u, wt))) { ok = false; break; }
           const uint32_t abase = smem_u32(sA + as * kAStageBytes);
           if (MODE == kModeFwd) {

@@ -3,6 +3,8 @@
 #include "qlora_nf4.h"
 
 #include <atomic>
+#include <chrono>
+#include <random>
 #include <cstring>
 #include <mutex>
 
@@ -241,12 +243,43 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
 int nn_proj(int r) { return (r + 15) / 16 * 16; }
 int64_t pad8(int64_t m) { return (m + 7) / 8 * 8; }
 
+// Last-wave split of one fused GEMM launch (see gemm_kernel.cuh): the tiles left for
+// the last round are split along the contraction when at most half the grid remains.
+struct GemmSplit {
+  int base = 0, count = 0;
+  size_t scratch_bytes() const { return static_cast<size_t>(count) * kWT * kBN * 4; }
+  size_t flag_bytes() const { return static_cast<size_t>(count) * 8; }
+};
+GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, int sms) {
+  GemmSplit g;
+  const int64_t tiles = ((M + kBN - 1) / kBN) * (n_out / kWT);
+  const int64_t grid = tiles < sms ? tiles : sms;
+  if (grid <= 0 || contraction / kBK < 2) return g;
+  const int64_t rem = tiles % grid;
+  if (rem > 0 && 2 * rem <= grid) {
+    g.base = static_cast<int>(tiles - rem);
+    g.count = static_cast<int>(rem);
+  }
+  return g;
+}
+size_t split_workspace(const GemmSplit &g) { return align256(g.scratch_bytes()) + align256(g.flag_bytes()); }
+
+// A value no flag left in a reused workspace can hold by chance: a per-process
+// random high half and a per-launch counter.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> ctr{
+      (static_cast<unsigned long long>(std::random_device{}()) << 32) |
+      static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count() & 0xFFFF0000ull)};
+  return ctr.fetch_add(1) + 1;
+}
+
 size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
   b += align256(static_cast<size_t>(N) * (K / 64) * 4);        // expanded block constants
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*XA hi/lo
   b += align256(static_cast<size_t>(M) * r * 4);               // XA when XA_out is NULL
+  b += split_workspace(gemm_split(M, N, K, sms));              // last-wave partial tiles
   return b + 256;
 }
 
@@ -259,6 +292,7 @@ size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*G hi/lo transposed
   b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*XA hi/lo transposed
   b += align256(static_cast<size_t>(M) * r * 4);               // XA recomputed
+  b += split_workspace(gemm_split(M, K, N, sms));              // last-wave partial tiles (dX)
   return b + 256;
 }
 
@@ -501,7 +535,7 @@ qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, 
 template <int MODE>
 qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, const float *S,
                          const uint16_t *lora_act_hl, const uint16_t *lora_w, int r,
-                         uint16_t *out, int sms, cudaStream_t st) {
+                         uint16_t *out, Workspace &ws, int sms, cudaStream_t st) {
   const int64_t N = Wq->rows, K = Wq->cols;
   const int64_t contraction = (MODE == kModeFwd) ? K : N;
   CUtensorMap tm_act, tm_codes, tm_scale, tm_lora;
@@ -541,6 +575,16 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, 
   std::memcpy(p.levels, T.levels, sizeof(p.levels));
   const int tiles = p.num_m_tiles * p.num_w_tiles;
   const int grid = tiles < sms ? tiles : sms;
+  const GemmSplit sp = gemm_split(M, (MODE == kModeFwd) ? N : K, contraction, sms);
+  p.split_base = sp.base;
+  p.split_count = sp.count;
+  p.kb_mid = p.kb_main / 2;
+  if (sp.count) {
+    p.scratch = static_cast<float *>(ws.take(sp.scratch_bytes()));
+    p.flags = static_cast<unsigned long long *>(ws.take(sp.flag_bytes()));
+    if (!p.scratch || !p.flags) return QLORA_ERR_WORKSPACE;
+    p.epoch = next_epoch();
+  }
   LaunchTimer lt(MODE == kModeFwd ? QLORA_K_GEMM_FWD : QLORA_K_GEMM_DX, st);
   qlora_gemm_kernel<MODE><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_scale,
                                                                       tm_lora, p);
@@ -699,7 +743,7 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
     fg.pending = false;
     if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
   }
-  return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, d->sms, stream);
+  return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, ws, d->sms, stream);
 }
 
 qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
@@ -756,7 +800,7 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
     fg.pending = false;
     if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
     lk.unlock();
-    if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, d->sms, stream)) != QLORA_OK) return st;
+    if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, ws, d->sms, stream)) != QLORA_OK) return st;
   }
   // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
   if ((st = launch_grad(X, M, K, ghlT, r, 0, dA, d->sms, stream)) != QLORA_OK) return st;

@@ -88,6 +88,8 @@ def _check(p, got, rows=None):
     (513, 256, 384, 64, 16.0),     # r=64: two LoRA stages
     (257, 128, 256, 128, 16.0),    # r=128: four LoRA stages
     (1000, 640, 896, 24, 48.0),    # r not a power of two
+    (300, 12800, 256, 16, 32.0),   # forward: 200 tiles on 148 CTAs, last round split in contraction halves
+    (300, 256, 12800, 16, 32.0),   # dX: the same split on the transposed GEMM
 ])
 def test_linear_fwd_bwd_full(q, M, N, K, r, alpha):
     p = linear_problem(M, N, K, r, alpha, 0.02, seed=0)
