@@ -659,7 +659,8 @@ qlora_status qlora_nf4_quantize(const uint16_t *W, int64_t rows, int64_t cols,
   const int64_t groups = (n + kGroupElems - 1) / kGroupElems;
   if (groups > 0x7FFFFFFFll) return QLORA_ERR_UNSUPPORTED_SHAPE;
   LaunchTimer lt(QLORA_K_QUANTIZE, stream);
-  const int64_t grid = groups < static_cast<int64_t>(d->sms) ? groups : static_cast<int64_t>(d->sms);
+  const int64_t ctas = static_cast<int64_t>(d->sms) * kQuantCtasPerSm;
+  const int64_t grid = groups < ctas ? groups : ctas;
   nf4_quantize_kernel<<<static_cast<unsigned>(grid > 0 ? grid : 1), kQuantThreads, kQuantSmemBytes, stream>>>(
       W, n, out->codes, out->q8, out->step, tab, static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull);
   return cuda_status(cudaGetLastError());

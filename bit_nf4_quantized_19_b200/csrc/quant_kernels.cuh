@@ -38,8 +38,8 @@ struct Levels {
 //   code:   bin j = round(32 xn) (exact, the low byte of 32 xn + 32 + 1.5*2^23 is
 //           j + 32), then code = bins[j].c + (xn > bins[j].t): the number of decision
 //           thresholds below xn, i.e. the nearest level with ties to the lower index.
-//           Every lane reads its own copy of the bin table (entry i of lane l at byte
-//           256 i + 8 l, one byte permute away from the sum), so the data-dependent
+//           Every lane of a half-warp reads its own copy of the bin table (entry i
+//           of copy c = lane mod 16 at byte 128 i + 8 c), so the data-dependent
 //           lookups never conflict on a bank;
 //   pack:   8 codes -> one 32-bit word (element 2j in the low nibble of byte j),
 //           accumulated as word = 16 word + code from the last element down;
@@ -67,6 +67,12 @@ QDEV void quotient_x2(float w0, float w1, float y, float neg_a, float &xn0, floa
       : "=f"(xn0), "=f"(xn1), "=f"(f0), "=f"(f1)
       : "f"(w0), "f"(w1), "f"(y), "f"(neg_a), "f"(32.0f), "f"(12582944.0f));
 }
+
+// Byte offset of bin entry i = (low byte of f) for this lane's table copy: entries
+// are 128-byte rows of 16 copies, copy (lane mod 16) at 8 (lane mod 16) = lane8.
+// A 64-bit shared load is served in two half-warp phases, so 16 copies keep every
+// data-dependent lookup conflict-free.
+QDEV uint32_t bin_offset(float f, uint32_t lane8) { return ((__float_as_uint(f) * 128u) & 0x7F80u) | lane8; }
 
 // max of two bf16x2 words, lane by lane, NaN-propagating
 QDEV uint32_t bmax2(uint32_t a, uint32_t b) {
@@ -143,8 +149,8 @@ QDEV void quant_compute(const uint4 (&v)[NP], int64_t n, int64_t gbase, int bl, 
       for (int j = 6; j >= 0; j -= 2) {
         float xa, xb, fa, fb;
         quotient_x2(w[j], w[j + 1], y, -a_b, xa, xb, fa, fb);
-        const uint2 tb = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(fb), lane8, 0x5504u));
-        const uint2 ta = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(fa), lane8, 0x5504u));
+        const uint2 tb = *reinterpret_cast<const uint2 *>(bins_bytes + bin_offset(fb, lane8));
+        const uint2 ta = *reinterpret_cast<const uint2 *>(bins_bytes + bin_offset(fa, lane8));
         // xn > t exactly when t - xn is negative (both finite; no threshold is zero,
         // so the difference is never a negative zero): its sign bit is the increment
         word = word * 16u + tb.y + (__float_as_uint(__fsub_rn(__uint_as_float(tb.x), xb)) >> 31);
@@ -165,7 +171,7 @@ QDEV void quant_compute(const uint4 (&v)[NP], int64_t n, int64_t gbase, int bl, 
           xn = __fdiv_rn(w[j], a);
         }
         const float f = __fmaf_rn(xn, 32.0f, 12582944.0f);
-        const uint2 t = *reinterpret_cast<const uint2 *>(bins_bytes + prmt(__float_as_uint(f), lane8, 0x5504u));
+        const uint2 t = *reinterpret_cast<const uint2 *>(bins_bytes + bin_offset(f, lane8));
         word = word * 16u + t.y + (xn > __uint_as_float(t.x) ? 1u : 0u);
       }
     }
@@ -182,28 +188,31 @@ QDEV void quant_compute(const uint4 (&v)[NP], int64_t n, int64_t gbase, int bl, 
   }
 }
 
-// One persistent CTA of 512 threads per SM.  The groups this CTA owns stream
-// through a ring of kQuantStages 32 KB buffers, each filled by one bulk copy on its
-// own mbarrier (kept kQuantStages groups ahead), so the SM always has about
-// 128 KB of loads in flight whatever the compute is doing; the compute reads its
-// 16-byte pieces from shared memory (consecutive threads, consecutive pieces).  The
-// one group that may end inside the tensor takes bounds-checked global loads.
+// Two persistent CTAs of 512 threads per SM (at most 64 registers per thread).  The
+// groups a CTA owns stream through a ring of kQuantStages 32 KB buffers, each filled
+// by one bulk copy on its own mbarrier (kept kQuantStages groups ahead), so the SM
+// always has about 128 KB of loads in flight whatever the compute is doing; the
+// compute reads its 16-byte pieces from shared memory (consecutive threads,
+// consecutive pieces).  The one group that may end inside the tensor takes
+// bounds-checked global loads.
 constexpr int kQuantThreads = 512;
-constexpr int kQuantStages = 4;
+constexpr int kQuantStages = 2;
+constexpr int kQuantCtasPerSm = 2;
+constexpr int kQuantCopies = 16;                                  // bin-table copies
 constexpr int kQuantPasses = kGroupElems / (kQuantThreads * 8);   // 4
 constexpr int kQuantStageBytes = kGroupElems * 2;                 // 32 KB
-constexpr int kQuantSmemBytes = kQuantStages * kQuantStageBytes + kQuantBins256 * 32 * 8 +
+constexpr int kQuantSmemBytes = kQuantStages * kQuantStageBytes + kQuantBins256 * kQuantCopies * 8 +
                                 (128 + kGroup + 16) * 4 + kQuantStages * 8 + 16;
 
-__global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(
+__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_kernel(
     const uint16_t *__restrict__ W, int64_t n, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ q8, float *__restrict__ step, const __grid_constant__ QuantTables tab,
     uint64_t limit_ns) {
   extern __shared__ __align__(128) uint8_t qsm[];
   uint8_t *ring = qsm;                                                             // [stages][32 KB]
   uint8_t *bins_bytes = qsm + kQuantStages * kQuantStageBytes;
-  uint2 *bins = reinterpret_cast<uint2 *>(bins_bytes);                             // [256 entries][32 lanes]
-  float *rcp = reinterpret_cast<float *>(bins_bytes + kQuantBins256 * 32 * 8);     // [128]
+  uint2 *bins = reinterpret_cast<uint2 *>(bins_bytes);                             // [256 entries][16 copies]
+  float *rcp = reinterpret_cast<float *>(bins_bytes + kQuantBins256 * kQuantCopies * 8);   // [128]
   float *amax = rcp + 128;                                                         // [256]
   float *wmax = amax + kGroup;                                                     // [16]
   uint64_t *full = reinterpret_cast<uint64_t *>(wmax + 16);                        // [stages]
@@ -214,8 +223,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(
   const int64_t G = gridDim.x;
   auto whole = [&](int64_t g) { return (g + 1) * kGroupElems <= n; };
 
-  for (int i = tid; i < kQuantBins256 * 32; i += kQuantThreads) {
-    const QuantBin e = tab.bins[i >> 5];
+  for (int i = tid; i < kQuantBins256 * kQuantCopies; i += kQuantThreads) {
+    const QuantBin e = tab.bins[i / kQuantCopies];
     bins[i] = make_uint2(__float_as_uint(e.t), static_cast<uint32_t>(e.c));
   }
   if (tid < 128) rcp[tid] = tab.rcp[tid];
@@ -232,7 +241,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(
     }
   }
   const Waiter waiter{abort_flag, limit_ns};
-  const uint32_t lane8 = 8u * static_cast<uint32_t>(lane);
+  const uint32_t lane8 = 8u * static_cast<uint32_t>(lane % kQuantCopies);
   const int sub = tid & 7;
   const int bl = tid >> 3;                     // block within a pass (0..63)
   bool nonfinite = false;
