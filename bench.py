@@ -395,9 +395,10 @@ def main():
            "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": e2e_steps, "uploads": "next step's inputs overlap the current step (two buffers)"}
 
-    # ---- HBM-bound subpaths (quantize / dequant of 1e9 values, skinny forward)
+    # ---- HBM-bound subpaths (quantize / dequant of 1e9 values, skinny forward): single-GPU
+    # measurements, taken at N = 1 only so a multi-GPU run stays short and symmetric
     subpaths = None
-    if not args.no_subpaths:
+    if not args.no_subpaths and world == 1:
         subpaths = hbm_subpaths(q, torch, dev, stream, P, flush)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
