@@ -19,6 +19,7 @@ import hashlib
 import json
 import os
 import statistics
+import tempfile
 import subprocess
 import sys
 import time
@@ -95,8 +96,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/qlora_clocks_{os.getpid()}.csv"
+        self.path = os.environ.get("QLORA_CLOCKS_CSV") or \
+            os.path.join(tempfile.gettempdir(), f"qlora_clocks_{os.getpid()}_gpu{gpu_index}.csv")
 
     def __enter__(self):
         try:
