@@ -125,6 +125,9 @@ qlora_status qlora_nf4_dequant(const qlora_nf4_t *Wq, uint16_t *W_out,
 /*
  * Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for an M-token
  * call on an N x K weight with LoRA rank r (the same size serves both calls).
+ * The size depends on the current device's SM count (the fused GEMM splits the
+ * tiles of its last round and keeps their partial sums here); query it on the
+ * device the calls will run on.
  */
 size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
@@ -135,6 +138,14 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * deq(W) is formed on chip in bf16, exactly as qlora_nf4_dequant, and never
  * written to memory.  Accumulation is fp32.  s = alpha / r.
  * Shapes: M >= 1; N % 128 == 0; K % 128 == 0; r % 8 == 0, 8 <= r <= 128.
+ * Execution: with M <= 16 tokens (and a contraction short enough for its
+ * shared-memory plan) the call takes the few-token path: X A in one small
+ * launch and the weight pass as its programmatic dependent.  Otherwise the
+ * block-constant expansion runs on a stream the library owns, forked from
+ * `stream` by an event record and joined back by an event wait before the
+ * GEMM.  Either way all work is ordered after what `stream` already holds and
+ * before what is enqueued to `stream` later, and the call can be captured into
+ * a CUDA graph.
  */
 qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
                               const uint16_t *A, const uint16_t *B, int r, float s,
@@ -154,7 +165,8 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
  * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - Returns QLORA_ERR_WORKSPACE, before launching anything, when the call
  *     needs more scratch than that (the need grows with M, N*K/16 and r;
- *     4096 tokens on an 11008 x 4096 weight with r = 16 needs about 5 MB).
+ *     4096 tokens on an 11008 x 4096 weight with r = 16 needs about 9 MB; at
+ *     r = 16 the first calls that do not fit come at about 36 k tokens).
  *   - The first call on each device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture on the device.
@@ -171,7 +183,9 @@ qlora_status qlora_linear_fwd_noalloc(const uint16_t *X, int64_t M, const qlora_
 
 /*
  * Backward of the adapted linear layer ([STEPS] Step 6: gradients flow through
- * the dequantized weights into the adapters; W is frozen, no dW):
+ * the dequantized weights into the adapters; W is frozen, no dW).  Ordering and
+ * graph capture as qlora_linear_fwd (the block-constant expansion for dX runs on
+ * the library's stream between a fork and a join on `stream`):
  *   G  = dY B^T                   (fp32 [M, r], internal)
  *   dX = dY deq(W) + s * G A^T    (bf16 [M, K]; skipped when dX is NULL)
  *   dA = s * X^T G                (fp32 [K, r])
