@@ -6,6 +6,7 @@
 #include <chrono>
 #include <random>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "common.cuh"
@@ -218,25 +219,77 @@ struct LmGeom {
   uint32_t tmem_cols;
 };
 
+// Clusters of one rank-r configuration the GPU holds at once (0 if the runtime cannot
+// say).  Cluster placement is per GPC, so this is well below sms * CTAs-per-SM / splits
+// for large shared-memory rings; the answer is cached per configuration.
+template <bool A_MN>
+int lm_max_clusters(int splits, int smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair(splits, smem);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(1, static_cast<unsigned>(splits), 1);
+  cfg.blockDim = dim3(kLmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, lora_mma_kernel<A_MN>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cache[key] = n;
+  return n;
+}
+
+// Split count and ring depth: the fewest waves of clusters, then the most splits (more
+// CTAs streaming the activation at once), then the deepest ring.  Each extra wave costs
+// a CTA's whole fixed latency (setup, first load, cluster reduction), which at these
+// sizes is as long as its streaming.
+template <bool A_MN>
 LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   LmGeom g{};
   g.nn = nn;
   g.row_tiles = static_cast<int>((rows + kLmRows - 1) / kLmRows);
   g.stages_total = static_cast<int>((contraction + 63) / 64);
-  int want = (2 * sms + g.row_tiles - 1) / g.row_tiles;
-  if (want < 1) want = 1;
-  if (want > kLmMaxSplits) want = kLmMaxSplits;     // the splits of a tile form one cluster
-  if (want > g.stages_total) want = g.stages_total;
-  g.sps = (g.stages_total + want - 1) / want;
-  g.splits = (g.stages_total + g.sps - 1) / g.sps;
-  int st = (110 * 1024) / (kLmABytes + nn * 128);
-  // the operand ring also holds the fp32 partial tile after the main loop
-  const int st_min = (kLmRows * nn * 4 + kLmABytes + nn * 128 - 1) / (kLmABytes + nn * 128);
-  if (st < st_min) st = st_min;
-  g.num_stages = st < 2 ? 2 : (st > 8 ? 8 : st);
   uint32_t tc = 32;
   while (tc < static_cast<uint32_t>(nn)) tc <<= 1;
   g.tmem_cols = tc;
+  const int stage_bytes = kLmABytes + nn * 128;
+  // the operand ring also holds the fp32 partial tile after the main loop
+  int st_min = (kLmRows * nn * 4 + stage_bytes - 1) / stage_bytes;
+  if (st_min < 3) st_min = 3;
+  int st_max = (110 * 1024) / stage_bytes;
+  if (st_max > 8) st_max = 8;
+  if (st_max < st_min) st_max = st_min;
+  int64_t best_waves = -1;
+  for (int c = kLmMaxSplits; c >= 1; c >>= 1) {   // the splits of a tile form one cluster
+    if (c > 1 && c > g.stages_total) continue;
+    const int total = g.stages_total > 0 ? g.stages_total : 1;
+    const int sps = (total + c - 1) / c;
+    const int splits = (total + sps - 1) / sps;
+    for (int S = st_max; S >= st_min; --S) {
+      int active = lm_max_clusters<A_MN>(splits, lora_mma_smem_bytes(nn, S));
+      if (active <= 0) active = (2 * sms) / splits;   // the runtime could not say
+      if (active <= 0) continue;
+      const int64_t waves = (g.row_tiles + active - 1) / active;
+      if (best_waves < 0 || waves < best_waves) {
+        best_waves = waves;
+        g.sps = sps;
+        g.splits = splits;
+        g.num_stages = S;
+      }
+      if (waves == 1) break;   // a deeper ring that still fits in one wave is preferred
+    }
+  }
   return g;
 }
 
@@ -335,7 +388,7 @@ qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_
                              const uint16_t *qop, int64_t q_rows, int64_t q_cols, int64_t q_pitch,
                              int64_t rows, int64_t contraction, int nn, LoraMmaParams p, int sms,
                              cudaStream_t st) {
-  const LmGeom g = lm_geom(rows, contraction, nn, sms);
+  const LmGeom g = lm_geom<A_MN>(rows, contraction, nn, sms);
   CUtensorMap tm_act, tm_q;
   // act is [act_rows (tokens), act_cols (features)] row-major bf16
   if (!make_map_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, act_cols, act_rows, act_cols * 2,

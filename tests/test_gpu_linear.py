@@ -186,3 +186,38 @@ def test_fwd_bwd_capture_in_cuda_graph(q):
     for got, want in zip((Y, XA, dX, dA, dB), ref):
         assert torch.equal(got.view(torch.int16) if got.dtype == torch.bfloat16 else got.view(torch.int32),
                            want.view(torch.int16) if want.dtype == torch.bfloat16 else want.view(torch.int32))
+
+
+@pytest.mark.gpu
+def test_capture_before_any_eager_call(q):
+    """A shape whose launch geometry the library has not chosen yet (the cluster
+    occupancy is queried on first use) captures into a CUDA graph as its first call;
+    replays match a later eager call bit for bit."""
+    import torch
+    p = linear_problem(200, 640, 768, 24, 48.0, 0.02, seed=11)
+    X, A, B, dY = (H.bits_to_dev(v) for v in (p.X, p.A, p.B, p.dY))
+    Wq = q.nf4_quantize(H.bits_to_dev(p.W))
+    ws = q.make_workspace(p.M, p.N, p.K, p.r, X.device)
+    outs = [torch.empty(p.M, p.N, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(p.M, p.r, dtype=torch.float32, device="cuda"),
+            torch.empty(p.M, p.K, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(p.K, p.r, dtype=torch.float32, device="cuda"),
+            torch.empty(p.r, p.N, dtype=torch.float32, device="cuda")]
+
+    def step(Y, XA, dX, dA, dB):
+        q.linear_fwd(X, Wq, A, B, p.s, workspace=ws, Y=Y, XA=XA)
+        q.linear_bwd(dY, X, XA, Wq, A, B, p.s, workspace=ws, dX=dX, dA=dA, dB=dB)
+
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(*outs)
+    g.replay()
+    torch.cuda.synchronize()
+    ref = [torch.empty_like(t) for t in outs]
+    step(*ref)
+    torch.cuda.synchronize()
+    assert q.device_status() == (0, 0)
+    for got, want in zip(outs, ref):
+        assert torch.equal(got.view(torch.int16) if got.dtype == torch.bfloat16 else got.view(torch.int32),
+                           want.view(torch.int16) if want.dtype == torch.bfloat16 else want.view(torch.int32))
