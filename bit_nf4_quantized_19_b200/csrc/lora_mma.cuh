@@ -47,6 +47,13 @@ struct LoraMmaParams {
   uint64_t limit_ns;
 };
 
+constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of a tile
+
+// Row pitch (floats) of the fp32 partial tile staged for the cluster reduction: odd, so
+// that both a warp over 32 rows of one column and a warp along one row hit 32 distinct
+// shared-memory banks.
+inline __host__ __device__ int lm_partial_pitch(int nn) { return nn + 1; }
+
 inline int lora_mma_smem_bytes(int nn, int stages) {
   return 1024 + stages * (kLmABytes + nn * 128) + 256;
 }
@@ -152,7 +159,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const Waiter dw{&no_abort, p.limit_ns};
     const bool got = __all_sync(0xffffffffu, wait_bar(done, 0, dw) ? 1 : 0);
     tc_fence_after();
-    float *dst = reinterpret_cast<float *>(smem) + rl * p.nn;
+    const int pitch = lm_partial_pitch(p.nn);
+    float *dst = reinterpret_cast<float *>(smem) + rl * pitch;
     for (int c = 0; c < p.nn; c += 16) {
       uint32_t v[16];
       asm volatile(
@@ -165,11 +173,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       tmem_wait_ld();
       const bool keep = got && nst > 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        *reinterpret_cast<float4 *>(dst + c + 4 * j) =
-            keep ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < 16; ++j) dst[c + j] = keep ? __uint_as_float(v[j]) : 0.f;
     }
   }
   tc_fence_before();
@@ -188,22 +192,35 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const int r0 = rank * R, r1 = min(kLmRows, r0 + R);
     const int nr = max(0, r1 - r0);
     const uint32_t base = smem_u32(smem);
+    const int pitch = lm_partial_pitch(p.nn);
     for (int i = tid; i < nr * p.r; i += kLmThreads) {
       int rr, j;
       if (p.grad && p.layout == 0) { rr = i / p.r; j = i - rr * p.r; }   // j fastest: out[row][j]
       else { j = i / nr; rr = i - j * nr; }                               // row fastest
       const int rl = r0 + rr, row = row0 + rl;
       if (row >= p.rows) continue;
-      const uint32_t a = base + 4u * static_cast<uint32_t>(rl * p.nn + j);
+      const uint32_t a = base + 4u * static_cast<uint32_t>(rl * pitch + j);
+      // every rank's load is issued before the sum, which runs in rank order
+      float pa[kLmClusterMax];
+#pragma unroll
+      for (int qq = 0; qq < kLmClusterMax; ++qq)
+        pa[qq] = qq < p.splits ? ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) : 0.f;
       float v = 0.f;
       if (p.grad) {
         const uint32_t b = a + 4u * static_cast<uint32_t>(p.r);
-        for (int qq = 0; qq < p.splits; ++qq)
-          v += ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) + ld_dsmem_f32(map_rank(b, static_cast<uint32_t>(qq)));
+        float pb[kLmClusterMax];
+#pragma unroll
+        for (int qq = 0; qq < kLmClusterMax; ++qq)
+          pb[qq] = qq < p.splits ? ld_dsmem_f32(map_rank(b, static_cast<uint32_t>(qq))) : 0.f;
+#pragma unroll
+        for (int qq = 0; qq < kLmClusterMax; ++qq)
+          if (qq < p.splits) v += pa[qq] + pb[qq];
         if (p.layout == 0) p.out[static_cast<int64_t>(row) * p.r + j] = v;
         else p.out[static_cast<int64_t>(j) * p.rows + row] = v;
       } else {
-        for (int qq = 0; qq < p.splits; ++qq) v += ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq)));
+#pragma unroll
+        for (int qq = 0; qq < kLmClusterMax; ++qq)
+          if (qq < p.splits) v += pa[qq];
         if (p.out) p.out[static_cast<int64_t>(row) * p.r + j] = v;
         uint16_t h, l;
         split_hilo(p.s * v, h, l);

@@ -212,7 +212,7 @@ struct Workspace {
 };
 
 // ---- launch geometry of the rank-r contractions (lora_mma_kernel)
-constexpr int kLmMaxSplits = 8;
+constexpr int kLmMaxSplits = kLmClusterMax;
 
 struct LmGeom {
   int nn, row_tiles, stages_total, sps, splits, num_stages;
@@ -265,7 +265,7 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   g.tmem_cols = tc;
   const int stage_bytes = kLmABytes + nn * 128;
   // the operand ring also holds the fp32 partial tile after the main loop
-  int st_min = (kLmRows * nn * 4 + stage_bytes - 1) / stage_bytes;
+  int st_min = (kLmRows * lm_partial_pitch(nn) * 4 + stage_bytes - 1) / stage_bytes;
   if (st_min < 3) st_min = 3;
   int st_max = (110 * 1024) / stage_bytes;
   if (st_max > 8) st_max = 8;
