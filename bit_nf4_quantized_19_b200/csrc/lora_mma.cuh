@@ -16,6 +16,8 @@
 //   MN-major (gradients):   Act^T tile [128 features x 64 tokens] from X / dY
 //                           [tokens, features]: two TMA boxes {64 features, 64 tokens}
 // Q is always K-major [nn rows x 64 c], TMA box {64, nn}.
+// dA and dB contract over the same tokens, so one launch computes both: the row tiles
+// of the second follow those of the first on the grid.
 // Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 4..7 epilogue.
 #pragma once
 #include "common.cuh"
@@ -45,6 +47,13 @@ struct LoraMmaParams {
   int ldT;
   int layout;
   uint64_t limit_ns;
+  // A second gradient product in the same launch: row tiles [tiles0, gridDim.x) compute
+  // it from the second pair of tensor maps.  It shares the contraction, nn and the
+  // splits; it has its own rows, output and layout.  tiles0 = gridDim.x: none.
+  int tiles0;
+  int rows1;
+  float *out1;
+  int layout1;
 };
 
 constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of a tile
@@ -68,6 +77,7 @@ QDEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
 template <bool A_MN>
 __global__ void __launch_bounds__(kLmThreads, 1)
     lora_mma_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_act1, const __grid_constant__ CUtensorMap tm_q1,
                     const __grid_constant__ LoraMmaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -83,7 +93,13 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = blockIdx.x * kLmRows;
+  const bool second = static_cast<int>(blockIdx.x) >= p.tiles0;
+  const int row0 = (static_cast<int>(blockIdx.x) - (second ? p.tiles0 : 0)) * kLmRows;
+  const int rows = second ? p.rows1 : p.rows;
+  float *const out = second ? p.out1 : p.out;
+  const int layout = second ? p.layout1 : p.layout;
+  const CUtensorMap *const map_act = second ? &tm_act1 : &tm_act;
+  const CUtensorMap *const map_q = second ? &tm_q1 : &tm_q;
   const int split = blockIdx.y;
   const int st0 = split * p.stages_per_split;
   const int st1 = min(p.stages_total, st0 + p.stages_per_split);
@@ -106,8 +122,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   const Waiter wt{abort_flag, p.limit_ns};
 
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_act);
-    prefetch_tmap(&tm_q);
+    prefetch_tmap(map_act);
+    prefetch_tmap(map_q);
     uint32_t armed = 0, last = 0;
     int s = 0;
     uint32_t ph = 0;
@@ -116,12 +132,12 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       const int c0 = (st0 + i) * 64;
       mbar_arrive_expect_tx(&full[s], kLmABytes + b_bytes);
       if (A_MN) {
-        tma_load_2d(sA + s * kLmABytes, &tm_act, &full[s], row0, c0);
-        tma_load_2d(sA + s * kLmABytes + 8192, &tm_act, &full[s], row0 + 64, c0);
+        tma_load_2d(sA + s * kLmABytes, map_act, &full[s], row0, c0);
+        tma_load_2d(sA + s * kLmABytes + 8192, map_act, &full[s], row0 + 64, c0);
       } else {
-        tma_load_2d(sA + s * kLmABytes, &tm_act, &full[s], c0, row0);
+        tma_load_2d(sA + s * kLmABytes, map_act, &full[s], c0, row0);
       }
-      tma_load_2d(sB + s * b_bytes, &tm_q, &full[s], c0, 0);
+      tma_load_2d(sB + s * b_bytes, map_q, &full[s], c0, 0);
       armed |= 1u << s;
       last = (last & ~(1u << s)) | (ph << s);
       if (++s == S) { s = 0; ph ^= 1u; }
@@ -195,10 +211,10 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const int pitch = lm_partial_pitch(p.nn);
     for (int i = tid; i < nr * p.r; i += kLmThreads) {
       int rr, j;
-      if (p.grad && p.layout == 0) { rr = i / p.r; j = i - rr * p.r; }   // j fastest: out[row][j]
+      if (p.grad && layout == 0) { rr = i / p.r; j = i - rr * p.r; }     // j fastest: out[row][j]
       else { j = i / nr; rr = i - j * nr; }                               // row fastest
       const int rl = r0 + rr, row = row0 + rl;
-      if (row >= p.rows) continue;
+      if (row >= rows) continue;
       const uint32_t a = base + 4u * static_cast<uint32_t>(rl * pitch + j);
       // every rank's load is issued before the sum, which runs in rank order
       float pa[kLmClusterMax];
@@ -215,13 +231,13 @@ __global__ void __launch_bounds__(kLmThreads, 1)
 #pragma unroll
         for (int qq = 0; qq < kLmClusterMax; ++qq)
           if (qq < p.splits) v += pa[qq] + pb[qq];
-        if (p.layout == 0) p.out[static_cast<int64_t>(row) * p.r + j] = v;
-        else p.out[static_cast<int64_t>(j) * p.rows + row] = v;
+        if (layout == 0) out[static_cast<int64_t>(row) * p.r + j] = v;
+        else out[static_cast<int64_t>(j) * rows + row] = v;
       } else {
 #pragma unroll
         for (int qq = 0; qq < kLmClusterMax; ++qq)
           if (qq < p.splits) v += pa[qq];
-        if (p.out) p.out[static_cast<int64_t>(row) * p.r + j] = v;
+        if (out) out[static_cast<int64_t>(row) * p.r + j] = v;
         uint16_t h, l;
         split_hilo(p.s * v, h, l);
         if (p.hl) {

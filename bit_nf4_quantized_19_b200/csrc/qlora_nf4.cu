@@ -380,24 +380,50 @@ int grid_for(int64_t total, int sms) {
   return g < 1 ? 1 : static_cast<int>(g);
 }
 
+// One operand pair of a rank-r product: act [act_rows (tokens), act_cols (features)]
+// row-major bf16, q [q_rows, q_cols] bf16 with a row pitch of q_pitch elements, and the
+// number of output rows.
+struct LmOperands {
+  const uint16_t *act;
+  int64_t act_rows, act_cols;
+  const uint16_t *q;
+  int64_t q_rows, q_cols, q_pitch;
+  int64_t rows;
+};
+
+template <bool A_MN>
+bool lm_maps(const LmOperands &o, int nn, CUtensorMap *tm_act, CUtensorMap *tm_q) {
+  return make_map_2d(tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.act, o.act_cols, o.act_rows, o.act_cols * 2,
+                     64, A_MN ? 64 : kLmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.q, o.q_cols, o.q_rows, o.q_pitch * 2, 64,
+                     static_cast<uint32_t>(nn), CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // D[rows, nn] = act (K-major rows x c, or MN-major c x rows) * q^T, split over the
 // contraction inside clusters of g.splits CTAs that reduce in rank order; the final
 // outputs are written by the kernel (projection or gradient form, see LoraMmaParams).
+// With `second`, the same launch also computes a second gradient product over the same
+// contraction (p.out1 / p.layout1 set by the caller); its row tiles follow the first's.
 template <bool A_MN>
-qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_cols,
-                             const uint16_t *qop, int64_t q_rows, int64_t q_cols, int64_t q_pitch,
-                             int64_t rows, int64_t contraction, int nn, LoraMmaParams p, int sms,
-                             cudaStream_t st) {
-  const LmGeom g = lm_geom<A_MN>(rows, contraction, nn, sms);
-  CUtensorMap tm_act, tm_q;
-  // act is [act_rows (tokens), act_cols (features)] row-major bf16
-  if (!make_map_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, act_cols, act_rows, act_cols * 2,
-                   64, A_MN ? 64 : kLmRows, CU_TENSOR_MAP_SWIZZLE_128B))
-    return QLORA_ERR_CUDA;
-  if (!make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qop, q_cols, q_rows, q_pitch * 2, 64,
-                   static_cast<uint32_t>(nn), CU_TENSOR_MAP_SWIZZLE_128B))
-    return QLORA_ERR_CUDA;
-  p.rows = static_cast<int>(rows);
+qlora_status launch_lora_mma(const LmOperands &o, int64_t contraction, int nn, LoraMmaParams p, int sms,
+                             cudaStream_t st, const LmOperands *second = nullptr) {
+  const int64_t tiles0 = (o.rows + kLmRows - 1) / kLmRows;
+  const int64_t tiles1 = second ? (second->rows + kLmRows - 1) / kLmRows : 0;
+  const LmGeom g = lm_geom<A_MN>((tiles0 + tiles1) * kLmRows, contraction, nn, sms);
+  CUtensorMap tm_act, tm_q, tm_act1, tm_q1;
+  if (!lm_maps<A_MN>(o, nn, &tm_act, &tm_q)) return QLORA_ERR_CUDA;
+  if (second) {
+    if (!lm_maps<A_MN>(*second, nn, &tm_act1, &tm_q1)) return QLORA_ERR_CUDA;
+    p.rows1 = static_cast<int>(second->rows);
+  } else {
+    tm_act1 = tm_act;
+    tm_q1 = tm_q;
+    p.rows1 = static_cast<int>(o.rows);
+    p.out1 = p.out;
+    p.layout1 = p.layout;
+  }
+  p.tiles0 = static_cast<int>(tiles0);
+  p.rows = static_cast<int>(o.rows);
   p.nn = nn;
   p.stages_total = g.stages_total;
   p.stages_per_split = g.sps;
@@ -420,7 +446,7 @@ qlora_status launch_lora_mma(const uint16_t *act, int64_t act_rows, int64_t act_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   LaunchTimer lt(A_MN ? QLORA_K_GRAD : QLORA_K_PROJECT, st);
-  return cuda_status(cudaLaunchKernelEx(&cfg, lora_mma_kernel<A_MN>, tm_act, tm_q, p));
+  return cuda_status(cudaLaunchKernelEx(&cfg, lora_mma_kernel<A_MN>, tm_act, tm_q, tm_act1, tm_q1, p));
 }
 
 // XA = X A (or G = dY B^T): fp32 [M, r] plus hi/lo of s*result in [M, 2r] and/or [2r, pad8(M)].
@@ -435,7 +461,8 @@ qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const 
   p.hl = hl;
   p.hlT = hlT;
   p.ldT = static_cast<int>(pad8(M));
-  return launch_lora_mma<false>(act, M, C, qT, r, C, C, M, C, nn_proj(r), p, sms, st);
+  const LmOperands o{act, M, C, qT, r, C, C, M};
+  return launch_lora_mma<false>(o, C, nn_proj(r), p, sms, st);
 }
 
 qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *hlT, int sms,
@@ -446,15 +473,22 @@ qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *
   return cuda_status(cudaGetLastError());
 }
 
-// g = act^T * (hi + lo) over tokens: act [M, C] bf16, hlT [2r, pad8(M)]; out dA [C, r] or dB [r, C].
-qlora_status launch_grad(const uint16_t *act, int64_t M, int64_t C, const uint16_t *hlT, int r,
-                         int layout, float *out, int sms, cudaStream_t st) {
+// Both adapter gradients in one launch, each act^T * (hi + lo) over the M tokens:
+// dA [K, r] = X^T (s G) from X [M, K] and ghlT [2r, pad8(M)];
+// dB [r, N] = (s XA)^T dY from dY [M, N] and xahlT [2r, pad8(M)].
+qlora_status launch_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t K, int64_t N,
+                          const uint16_t *ghlT, const uint16_t *xahlT, int r, float *dA, float *dB,
+                          int sms, cudaStream_t st) {
   LoraMmaParams p{};
   p.grad = 1;
   p.r = r;
-  p.out = out;
-  p.layout = layout;
-  return launch_lora_mma<true>(act, M, C, hlT, 2 * r, M, pad8(M), C, M, 2 * r, p, sms, st);
+  p.out = dA;
+  p.layout = 0;
+  p.out1 = dB;
+  p.layout1 = 1;
+  const LmOperands a{X, M, K, ghlT, 2 * r, M, pad8(M), K};
+  const LmOperands b{dY, M, N, xahlT, 2 * r, M, pad8(M), N};
+  return launch_lora_mma<true>(a, M, 2 * r, p, sms, st, &b);
 }
 
 qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT, int sms, cudaStream_t st) {
@@ -857,8 +891,7 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
     if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, ws, d->sms, stream)) != QLORA_OK) return st;
   }
   // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
-  if ((st = launch_grad(X, M, K, ghlT, r, 0, dA, d->sms, stream)) != QLORA_OK) return st;
-  return launch_grad(dY, M, N, xahlT, r, 1, dB, d->sms, stream);
+  return launch_grads(X, dY, M, K, N, ghlT, xahlT, r, dA, dB, d->sms, stream);
 }
 
 qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags) {
