@@ -237,7 +237,8 @@ typedef enum {
   QLORA_K_PROJECT = 3,      /* XA = X A or G = dY B^T (+ hi/lo)     */
   QLORA_K_GEMM_FWD = 4,     /* fused dequant GEMM, forward          */
   QLORA_K_GEMM_DX = 5,      /* fused dequant GEMM, dX               */
-  QLORA_K_GRAD = 6,         /* adapter gradients dA, dB             */
+  QLORA_K_GRAD = 6,         /* adapter gradients dA and dB (one     */
+                            /* launch computes both)                */
   QLORA_K_GRAD_REDUCE = 7,  /* unused: the split sums now happen    */
                             /* inside the QLORA_K_GRAD launches     */
   QLORA_K_SKINNY = 8        /* few-token forward                    */
