@@ -88,53 +88,107 @@ def traffic_for(kernel_key):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """nvidia-smi clocks and throttle reasons sampled every 20 ms while running.
+    Each sample carries nvidia-smi's own timestamp; summary() keeps the samples
+    taken between entering and leaving the block (the timed region).  If
+    nvidia-smi refuses that query, the sampler falls back to the same fields
+    without the timestamp every 200 ms, and summary() then uses every sample."""
+    BASIC = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    FIELDS = BASIC + ",timestamp"
+    INTERVAL_MS = 20
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.fh = None
+        self.t0 = self.t1 = None
+        self.interval = self.INTERVAL_MS
         self.path = os.environ.get("QLORA_CLOCKS_CSV") or \
             os.path.join(tempfile.gettempdir(), f"qlora_clocks_{os.getpid()}_gpu{gpu_index}.csv")
 
-    def __enter__(self):
+    def _start(self, fields, interval_ms):
+        """Start sampling.  False only if nvidia-smi is missing or exits within 3 s
+        (a refused query); a slow first sample is not a failure."""
+        self.interval = interval_ms
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={fields}",
+                 "--format=csv,noheader,nounits", "-lms", str(interval_ms)], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
         except Exception:
-            self.proc = None
-        time.sleep(0.3)
-        return self
+            self._stop()
+            return False
+        deadline = time.time() + 3.0
+        while time.time() < deadline:
+            if self.proc.poll() is not None:
+                self._stop()
+                return False
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
+        return True
 
-    def __exit__(self, *a):
+    def _stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            self.proc = None
+        if self.fh is not None:
             self.fh.close()
+            self.fh = None
+
+    def __enter__(self):
+        if not self._start(self.FIELDS, self.INTERVAL_MS):
+            self._start(self.BASIC, 200)
+        time.sleep(0.1)
+        self.t0 = time.time()
+        return self
+
+    def __exit__(self, *a):
+        self.t1 = time.time()
+        if self.proc is not None:
+            time.sleep(2 * self.interval / 1000.0)
+        self._stop()
+
+    @staticmethod
+    def _stamp(text):
+        import datetime
+        return datetime.datetime.strptime(text.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
 
     def summary(self):
         try:
             rows = [l.strip().split(", ") for l in open(self.path) if l.strip()]
         except Exception:
             return None
+        rows = [r for r in rows if len(r) >= 9]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4)
-                          if len(r) > 5 + i and r[5 + i].strip().lower() == "active"})
+        window = None
+        if self.t0 is not None and self.t1 is not None:
+            try:
+                lo, hi = self.t0 - self.interval / 1000.0, self.t1 + self.interval / 1000.0
+                inside = [r for r in rows if len(r) >= 10 and lo <= self._stamp(r[9]) <= hi]
+                window = inside
+            except Exception:
+                window = None
+        use = window if window else rows
+        sm = [float(r[1]) for r in use if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in use if r[2].replace(".", "").isdigit()]
+        watts = [float(r[3]) for r in use if r[3].replace(".", "").isdigit()]
+        reasons = sorted({self.REASONS[i] for r in use for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(use), "in_timed_region": bool(window),
+                "power_w": statistics.median(watts) if watts else None,
+                "interval_ms": self.interval}
 
 
 # ------------------------------------------------------------------ oracle baseline
