@@ -92,3 +92,23 @@ def test_argument_errors_before_any_launch(L):
 def test_wait_limit_setter_roundtrip(L):
     old = L.qlora_set_wait_limit_us(123)
     assert L.qlora_set_wait_limit_us(old) == 123
+
+
+def test_plain_c_consumer(L, tmp_path):
+    """tests/csrc/abi_consumer.c: a C11 program built with gcc against the header
+    alone (-Wall -Wextra -pedantic -Werror) and linked to the shared library runs
+    the host-side checks; its exit status is its number of failed checks."""
+    import os
+    import subprocess
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    pkg = os.path.dirname(build.LIB_PATH)
+    exe = str(tmp_path / "abi_consumer")
+    cc = subprocess.run(["gcc", "-std=c11", "-O1", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(root, "include"), os.path.join(here, "csrc", "abi_consumer.c"),
+                         "-L", pkg, "-lqlora_nf4", f"-Wl,-rpath,{pkg}", "-lm", "-o", exe],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stderr
+    assert "all checks passed" in run.stdout
