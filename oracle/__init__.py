@@ -24,6 +24,10 @@ on 32-bit values):
 * ``linear.forward`` / ``linear.backward`` -- Y = X deq(W)^T + s (X A) B and its
   gradients for X, A, B (W frozen), accumulated in fp64.  Sources:
   ozercemkelahmet.com, How it works, Steps 5-6.
+* ``linear.merge_weight`` -- the adapter folded into a 16-bit weight,
+  bf16(W_base + s (A B)^T), rounded once from the fp64 sum
+  (``nf4.f64_to_bf16_rn``).  Sources: ozercemkelahmet.com, How it works, Step 8,
+  section "Merging after QLoRA", and its FAQ on merging.
 
 Readings taken where the pages are silent (each one is listed with its reason in
 the design notes of the repository):

@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .nf4 import bf16_to_f32
+from .nf4 import bf16_to_f32, f64_to_bf16_rn
 
 
 def as_f64(bits_or_f) -> np.ndarray:
@@ -67,6 +67,22 @@ def backward_rows_dx(dY, Wd, A, B, s: float, rows):
     Wd, A, B = (as_f64(t) for t in (Wd, A, B))
     G = dY @ B.T
     return dY @ Wd + s * (G @ A.T)
+
+
+def merge_weight(W_base, A, B, s: float) -> np.ndarray:
+    """The adapter folded into a 16-bit weight for serving ("QLoRA",
+    ozercemkelahmet.com, How it works, Step 8 and section "Merging after QLoRA";
+    its FAQ on merging): W_merged = W_base + s (A B)^T, stored in bf16.
+
+    W_base [N, K] is the 16-bit original or the dequantized NF4 weight (the
+    pages prefer the original and allow the dequantized copy), as bf16 bits;
+    A [K, r], B [r, N] bf16 bits.  The sum is exact in fp64 up to its own
+    rounding and is rounded once to bf16 (nearest, ties to even).  With this,
+    Y = X W_merged^T equals the adapted forward up to that rounding.
+    Returns bf16 bits [N, K].
+    """
+    Wb, A, B = (as_f64(t) for t in (W_base, A, B))
+    return f64_to_bf16_rn(Wb + s * (A @ B).T)
 
 
 def rel_fro(got, ref) -> float:

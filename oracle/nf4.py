@@ -72,6 +72,37 @@ def f32_to_bf16_rn(x: np.ndarray) -> np.ndarray:
     return out.astype(np.uint16)
 
 
+def f64_to_bf16_rn(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to bf16 in ONE step, nearest, ties to even, as bits.
+
+    Going through float32 first would round twice, which differs from one
+    rounding when the fp32 step lands exactly on a bf16 tie.  Same plain
+    definition as above, on the exact fp64 value: the bf16 quantum at x is
+    2^(e-8) for x = m 2^e, m in [0.5, 1) (2^-133 below the normal range); the
+    two neighbours are x truncated to a multiple of it and the next multiple
+    away from zero; the nearer wins, a tie goes to the one with an even last
+    bit.  Magnitudes that round to 2^128 or beyond give infinity.  Finite
+    inputs only.
+    """
+    x = np.asarray(x, np.float64)
+    shape = x.shape
+    x = x.ravel()
+    _, e = np.frexp(x)
+    e = np.maximum(e, -125)                      # below 2^-126 the quantum stays 2^-133
+    q = np.ldexp(1.0, e - 8)
+    t = np.trunc(x / q)                          # exact: x / q only shifts the exponent
+    lo = t * q
+    hi = (t + np.sign(x)) * q
+    d_lo = np.abs(x - lo)
+    d_hi = np.abs(hi - x)
+    lo_even = np.mod(np.abs(t), 2) == 0
+    v = np.where((d_hi < d_lo) | ((d_hi == d_lo) & ~lo_even), hi, lo)
+    v = np.where(np.abs(v) >= 2.0 ** 128, np.copysign(np.inf, x), v)
+    v = np.where(x == 0, x, v)                   # keeps the sign of a zero
+    bits = (v.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    return bits.reshape(shape)
+
+
 # ---------------------------------------------------------------------------
 # a2: block absmax
 # ---------------------------------------------------------------------------
