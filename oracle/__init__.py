@@ -28,6 +28,15 @@ on 32-bit values):
   bf16(W_base + s (A B)^T), rounded once from the fp64 sum
   (``nf4.f64_to_bf16_rn``).  Sources: ozercemkelahmet.com, How it works, Step 8,
   section "Merging after QLoRA", and its FAQ on merging.
+* ``nf4.quantize_single_level`` / ``nf4.dequantize_single_level`` -- Steps 1-2
+  without Step 3: the same codes, the block constants kept in fp32 (half a bit
+  per weight).  Source: ozercemkelahmet.com, How it works, Step 2.
+* ``linear.forward_dropout`` / ``linear.backward_dropout`` /
+  ``linear.accumulate_grads`` -- inverted dropout of the adapter input with a
+  caller-drawn keep mask, and dA / dB summed over micro-batches.  Sources:
+  ozercemkelahmet.com, "A code example with common libraries" (lora_dropout),
+  "Training arguments" (gradient_accumulation_steps) and "Reading the memory
+  profile".
 
 Readings taken where the pages are silent (each one is listed with its reason in
 the design notes of the repository):

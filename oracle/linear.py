@@ -85,6 +85,46 @@ def merge_weight(W_base, A, B, s: float) -> np.ndarray:
     return f64_to_bf16_rn(Wb + s * (A @ B).T)
 
 
+def dropout_input(X, keep, p: float) -> np.ndarray:
+    """Inverted dropout of the adapter input: X * keep / (1 - p), fp64.  `keep` is
+    the 0/1 mask (drawn by the caller, Bernoulli(1 - p) per element); the frozen
+    path still sees the undropped X."""
+    return as_f64(X) * (np.asarray(keep, np.float64) / (1.0 - p))
+
+
+def forward_dropout(X, Wd, A, B, s: float, keep, p: float):
+    """Y = X Wd^T + s (drop(X) A) B with drop the inverted dropout above: the
+    adapter input dropout of a LoRA configuration ("QLoRA", ozercemkelahmet.com,
+    "A code example with common libraries", lora_dropout)."""
+    Xd = dropout_input(X, keep, p)
+    XA = Xd @ as_f64(A)
+    Y = as_f64(X) @ as_f64(Wd).T + s * (XA @ as_f64(B))
+    return Y, XA
+
+
+def backward_dropout(dY, X, Wd, A, B, s: float, keep, p: float, XA=None):
+    """Gradients of forward_dropout for a fixed mask: G = dY B^T;
+    dX = dY Wd + s (G A^T) * keep / (1 - p);  dA = s drop(X)^T G;
+    dB = s XA^T dY with XA = drop(X) A."""
+    dY, Wd, A, B = (as_f64(t) for t in (dY, Wd, A, B))
+    Xd = dropout_input(X, keep, p)
+    XA = Xd @ A if XA is None else np.asarray(XA, np.float64)
+    G = dY @ B.T
+    dX = dY @ Wd + s * (G @ A.T) * (np.asarray(keep, np.float64) / (1.0 - p))
+    return dict(G=G, dX=dX, dA=s * (Xd.T @ G), dB=s * (XA.T @ dY))
+
+
+def accumulate_grads(acc: dict | None, grads: dict) -> dict:
+    """Gradient accumulation over micro-batches ("QLoRA", ozercemkelahmet.com,
+    "Training arguments", gradient_accumulation_steps; "Reading the memory
+    profile": smaller micro-batches with more accumulation steps keep the
+    effective batch): dA and dB are summed over the micro-batches before the
+    optimizer step."""
+    if acc is None:
+        return {k: np.array(grads[k], np.float64) for k in ("dA", "dB")}
+    return {k: acc[k] + grads[k] for k in ("dA", "dB")}
+
+
 def rel_fro(got, ref) -> float:
     """||got - ref||_F / ||ref||_F."""
     got = np.asarray(got, np.float64)

@@ -246,3 +246,34 @@ def dequantize(packed, q8, step, n: int) -> np.ndarray:
     scale = np.repeat(block_scales(q8, step), BLOCK)[:n]
     prod = (L[codes] * scale).astype(np.float32)
     return f32_to_bf16_rn(prod)
+
+
+# ---------------------------------------------------------------------------
+# single-level variant: Steps 1-2 without Step 3
+# ---------------------------------------------------------------------------
+def storage_bytes_single_level(n: int):
+    """Bytes of (packed codes, fp32 block constants) when the block constants are
+    kept in fp32 ("QLoRA", ozercemkelahmet.com, How it works, Step 2: one 32-bit
+    constant per 64 values, half a bit per weight)."""
+    nb = (n + BLOCK - 1) // BLOCK
+    return (n + 1) // 2, 4 * nb
+
+
+def quantize_single_level(w) -> dict:
+    """Blockwise NF4 with fp32 block constants (no double quantization): the
+    codes of Steps 1-2, which use the unquantized absmax exactly as quantize()
+    does, and the absmax itself as the stored constant."""
+    w = np.asarray(w, np.float32).ravel()
+    a = block_absmax(w)
+    codes = block_codes(w, a)
+    return dict(n=w.size, codes=pack_codes(codes), absmax=a, codes_unpacked=codes)
+
+
+def dequantize_single_level(packed, absmax, n: int) -> np.ndarray:
+    """bf16 bits of bf16_RN(RN32(L[code] * a_b)): the level times the block's
+    stored fp32 constant, into the bf16 compute type."""
+    codes = unpack_codes(packed, n)
+    L = nf4_levels()
+    scale = np.repeat(np.asarray(absmax, np.float32).ravel(), BLOCK)[:n]
+    prod = (L[codes] * scale).astype(np.float32)
+    return f32_to_bf16_rn(prod)
