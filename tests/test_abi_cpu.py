@@ -112,3 +112,43 @@ def test_plain_c_consumer(L, tmp_path):
     run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, run.stderr
     assert "all checks passed" in run.stdout
+
+
+def _c_kind(decl: str) -> str:
+    d = " ".join(decl.split())
+    if "*" in d or "[" in d or d.startswith("qlora_stream_t"):
+        return "ptr"
+    for prefix, kind in (("int64_t", "i64"), ("uint32_t", "u32"), ("size_t", "sz"), ("float", "f32"),
+                         ("qlora_status", "int"), ("int", "int")):
+        if d == prefix or d.startswith(prefix + " "):
+            return kind
+    raise AssertionError(f"unknown C type in {decl!r}")
+
+
+def _py_kind(t) -> str:
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(t, type(ctypes.POINTER(ctypes.c_int))):
+        return "ptr"
+    for ct, kind in ((ctypes.c_int64, "i64"), (ctypes.c_uint32, "u32"), (ctypes.c_size_t, "sz"),
+                     (ctypes.c_float, "f32"), (ctypes.c_int, "int")):
+        if t is ct:
+            return kind
+    raise AssertionError(f"unknown ctypes type {t!r}")
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype in include/qlora_nf4.h has the same return type and the same
+    parameter count and kinds (pointer, int64, int, uint32, size_t, float) as its
+    ctypes declaration, so the binding cannot drift from the C ABI."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(_abi.HEADER).read(), flags=re.S)
+    protos = re.findall(r"([A-Za-z_][\w \t\*]*?)\b(qlora_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert len(protos) == len(_abi.SIGNATURES)
+    for ret, name, params in protos:
+        res, args = _abi.SIGNATURES[name]
+        ret = " ".join(ret.split())
+        want_ret = "void" if ret == "void" else _c_kind(ret)
+        assert _py_kind(res) == want_ret, (name, ret, res)
+        plist = [] if params.strip() in ("", "void") else params.split(",")
+        assert [_c_kind(p) for p in plist] == [_py_kind(a) for a in args], name
