@@ -87,6 +87,17 @@ def traffic_for(kernel_key):
     return None
 
 
+def smi_device_id(local: int, visible: str | None) -> str:
+    """nvidia-smi's --id for CUDA device `local`: its entry in CUDA_VISIBLE_DEVICES
+    (a physical index or a GPU UUID, both of which nvidia-smi accepts), else the
+    index itself."""
+    if visible:
+        ids = [v.strip() for v in visible.split(",") if v.strip()]
+        if 0 <= local < len(ids) and (ids[local].isdigit() or ids[local].startswith("GPU-")):
+            return ids[local]
+    return str(local)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 20 ms while running.
     Each sample carries nvidia-smi's own timestamp; summary() keeps the samples
@@ -116,7 +127,8 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={fields}",
+                ["nvidia-smi", f"--id={smi_device_id(self.gpu, os.environ.get('CUDA_VISIBLE_DEVICES'))}",
+                 f"--query-gpu={fields}",
                  "--format=csv,noheader,nounits", "-lms", str(interval_ms)], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
         except Exception:

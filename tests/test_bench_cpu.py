@@ -135,3 +135,13 @@ def test_clock_sampler_process_paths(tmp_path, monkeypatch, mode):
         assert c.interval == 200 and got["in_timed_region"] is False and got["samples"] >= 1
     else:
         assert c.interval == 20 and got is None
+
+
+def test_smi_device_id_follows_cuda_visible_devices():
+    assert bench.smi_device_id(0, None) == "0"
+    assert bench.smi_device_id(1, "3,5") == "5"
+    assert bench.smi_device_id(0, "GPU-0a1b2c3d-0000-1111-2222-333344445555") == \
+        "GPU-0a1b2c3d-0000-1111-2222-333344445555"
+    assert bench.smi_device_id(2, "3,5") == "2"          # out of range: the index itself
+    assert bench.smi_device_id(0, "all") == "0"          # not an index or a UUID
+    assert bench.smi_device_id(0, "") == "0"
