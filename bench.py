@@ -1,13 +1,16 @@
 #!/usr/bin/env python
 """Benchmark of the QLoRA NF4 frozen-base linear layer on B200.
 
-One step = forward + backward of the three LLaMA-7B-shaped adapted projections
-(W 4096x4096, 11008x4096, 4096x11008 stored as NF4 with double-quantized
-constants; 4096 tokens per GPU; LoRA r=16, alpha=32): per projection
-Y = X deq(W)^T + s (X A) B, then dX, dA, dB.  Weights are quantized once before
-timing (model load).  Metric: fwd+bwd TFLOP/s of algorithmic FLOPs
-4MNK + 6Mr(K+N) per projection.  Multi-GPU: data-parallel replicas (weak
-scaling), each rank its own 4096 tokens, dA/dB all-reduced over NCCL each step.
+One step = forward + backward of the adapted projections of one workload, each
+Y = X deq(W)^T + s (X A) B followed by dX, dA and dB, with the weights stored as
+NF4 with double-quantized constants and quantized once before timing (model
+load).  The headline workload is the largest single-GPU one: the three
+LLaMA-65B-shaped projections W 8192x8192, 22016x8192 and 8192x22016 with 8192
+tokens per GPU, LoRA r = 64, alpha = 16.  The LLaMA-7B-shaped projections (4096
+tokens, r = 16) and the small single layer (16 tokens on W 1024x1024, reported in
+microseconds) are measured after it.  Metric: fwd+bwd TFLOP/s of the algorithmic
+FLOPs 4MNK + 6Mr(K+N) per projection.  Multi-GPU: data-parallel replicas (weak
+scaling), each rank its own tokens, dA/dB all-reduced over NCCL each step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -29,15 +32,25 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from synth import WORKLOADS  # noqa: E402  (shapes and distributions of every workload)
+
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4-weight HBM GB/s vs roofline, 1 B200"
-SHAPES = [(4096, 4096, 4096), (4096, 11008, 4096), (4096, 4096, 11008)]   # (M, N, K)
-RANK_R, ALPHA, W_STD = 16, 32.0, 0.02
-WORKLOAD = ("LLaMA-7B-shaped projections W[N,K] in {4096x4096, 11008x4096, 4096x11008}, NF4 "
-            "block 64 / double-quant 256; 4096 tokens per GPU; LoRA r=16 alpha=32; fwd+bwd")
+HEADLINE = "llama65b"
+WORKLOAD_TEXT = {
+    "llama65b": ("LLaMA-65B-shaped projections W[N,K] in {8192x8192, 22016x8192, 8192x22016}, NF4 "
+                 "block 64 / double-quant 256, W ~ N(0,0.015); 8192 tokens per GPU; LoRA r=64 "
+                 "alpha=16; fwd+bwd"),
+    "llama7b": ("LLaMA-7B-shaped projections W[N,K] in {4096x4096, 11008x4096, 4096x11008}, NF4 "
+                "block 64 / double-quant 256, W ~ N(0,0.02); 4096 tokens per GPU; LoRA r=16 alpha=32; "
+                "fwd+bwd"),
+    "small": "single QLoRA linear W 1024x1024 NF4, 16 tokens, LoRA r=8 alpha=16; fwd+bwd",
+}
+WORKLOAD = WORKLOAD_TEXT[HEADLINE]
 FLUSH_BYTES = 256 << 20
 SKINNY = [(m, n, 4096) for n in (4096, 11008) for m in (1, 4, 16)]
 BIG_N = 1_000_000_000
 GRAPH_STREAM_BYTES = 320 << 20   # weights streamed per graph replay of the decode measurement
+SMALL_CALLS = 50
 
 
 def step_flops(M, N, K, r):
@@ -49,9 +62,10 @@ def peaks():
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
         return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
-                    bf16_sus=float(p["bf16_tflops_sustained"]), src="measured")
+                    bf16_sus=float(p["bf16_tflops_sustained"]), sm_max_mhz=p.get("sm_max_mhz"),
+                    src="measured")
     except Exception:
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max_mhz=1965.0, src="fallback")
 
 
 def source_hash(kernel_key):
@@ -204,6 +218,20 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle baseline
+def sample_problems(name, tokens, wrows):
+    """The leading part of every projection of a workload, bit-identical to what the
+    GPU arm runs on: the first `wrows` output features (rows of W) and the first
+    `tokens` tokens; A and B whole."""
+    from synth import linear_problem_rows
+    wl = WORKLOADS[name]
+    out = []
+    for (M, N, K) in wl["shapes"]:
+        p = linear_problem_rows(M, N, K, wl["r"], wl["alpha"], wl["w_std"], tokens, wrows, seed=0)
+        out.append(dict(M=M, N=N, K=K, r=wl["r"], s=wl["alpha"] / wl["r"], W=p.W, X=p.X, A=p.A,
+                        B=p.B, dY=p.dY))
+    return out
+
+
 def oracle_sample(problems, tokens, wrows, repeats=1):
     """Oracle fwd+bwd on a bounded sample of every projection: the first
     `tokens` tokens and the first `wrows` output features (dequant of those W
@@ -236,24 +264,46 @@ def cpu_info():
     return cores, blas
 
 
-def host_problems(seed):
-    from synth import linear_problem
+def host_problems(name, rank=0):
+    """Seeded inputs of one workload (bf16 bits on the host).  The frozen W, A and B
+    are the same on every rank; X and dY are each rank's own tokens."""
+    from synth import linear_problem, normal_bf16
+    wl = WORKLOADS[name]
+    r, alpha, w_std = wl["r"], wl["alpha"], wl["w_std"]
     out = []
-    for (M, N, K) in SHAPES:
-        p = linear_problem(M, N, K, RANK_R, ALPHA, W_STD, seed=0)      # frozen W: same on all ranks
-        if seed:
-            q = linear_problem(M, N, K, RANK_R, ALPHA, W_STD, seed=seed)
-            p.X, p.dY = q.X, q.dY                                      # per-rank tokens
-        out.append(dict(M=M, N=N, K=K, r=RANK_R, s=ALPHA / RANK_R, W=p.W, X=p.X, A=p.A, B=p.B,
-                        dY=p.dY))
+    for (M, N, K) in wl["shapes"]:
+        p = linear_problem(M, N, K, r, alpha, w_std, seed=0)
+        X, dY = p.X, p.dY
+        if rank:
+            X = normal_bf16(rank, f"X{M}x{N}x{K}r{r}", (M, K), 1.0)
+            dY = normal_bf16(rank, f"dY{M}x{N}x{K}r{r}", (M, N), 1.0)
+        out.append(dict(M=M, N=N, K=K, r=r, s=alpha / r, W=p.W, X=X, A=p.A, B=p.B, dY=dY))
     return out
+
+
+def workload_flops(name):
+    wl = WORKLOADS[name]
+    return sum(step_flops(M, N, K, wl["r"]) for (M, N, K) in wl["shapes"])
+
+
+def gemm_flops(name):
+    """FLOPs of the fused GEMM launches of one step: forward 2MNK + 2MNr (its LoRA
+    K-steps), dX 2MNK + 2MKr."""
+    wl = WORKLOADS[name]
+    r = wl["r"]
+    return sum(4.0 * M * N * K + 2.0 * M * N * r + 2.0 * M * K * r for (M, N, K) in wl["shapes"])
+
+
+# the bounded oracle samples: (tokens, output features) of every projection
+CPU_SAMPLE = {"llama65b": (256, 1024), "llama7b": (512, 2048)}
+REF_SAMPLE = {"llama65b": (64, 256)}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    problems = host_problems(0)
-    tokens, wrows = 128, 512
+    tokens, wrows = REF_SAMPLE[HEADLINE]
+    problems = sample_problems(HEADLINE, tokens, wrows)
     for _ in range(max(0, args.warmup)):
         oracle_sample(problems, tokens, wrows)
     fl, t = 0.0, 0.0
@@ -278,16 +328,239 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+class Workload:
+    """Device-resident state of one workload: quantized weights, inputs, outputs,
+    workspaces, the gradient bucket and pinned host copies of the inputs."""
+
+    def __init__(self, q, torch, dev, name, rank, pinned=True):
+        from bit_nf4_quantized_19_b200.dp import GradBucket
+        self.q, self.torch, self.dev, self.name = q, torch, dev, name
+        wl = WORKLOADS[name]
+        self.shapes = wl["shapes"]
+        self.r = wl["r"]
+        hp = host_problems(name, rank)
+        self.bucket = GradBucket([(N, K, self.r) for (_, N, K) in self.shapes], dev)
+        self.layers = []
+
+        def to_dev(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        def to_pinned(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        for p, (dA, dB) in zip(hp, self.bucket.views):
+            M, N, K, r = p["M"], p["N"], p["K"], p["r"]
+            L = dict(M=M, N=N, K=K, r=r, s=p["s"], Wq=q.nf4_quantize(to_dev(p["W"])),
+                     X=to_dev(p["X"]), dY=to_dev(p["dY"]), A=to_dev(p["A"]), B=to_dev(p["B"]),
+                     Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                     XA=torch.empty(M, r, dtype=torch.float32, device=dev),
+                     dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+                     dA=dA, dB=dB, ws=q.make_workspace(M, N, K, r, dev))
+            if pinned:
+                L["hX"], L["hdY"] = to_pinned(p["X"]), to_pinned(p["dY"])
+            self.layers.append(L)
+        del hp
+        self.flops = workload_flops(name)
+        self.gemm_flops = gemm_flops(name)
+
+    def run(self, inputs=None):
+        """One fwd+bwd of every projection (optionally on other X / dY buffers), then
+        the one exchange of data-parallel adapter training."""
+        q = self.q
+        for i, L in enumerate(self.layers):
+            X, dY = (L["X"], L["dY"]) if inputs is None else inputs[i]
+            q.linear_fwd(X, L["Wq"], L["A"], L["B"], L["s"], workspace=L["ws"], Y=L["Y"], XA=L["XA"])
+            q.linear_bwd(dY, X, L["XA"], L["Wq"], L["A"], L["B"], L["s"],
+                         workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
+        self.bucket.allreduce_()
+
+
+def time_steps(torch, run, steps, flush, stream, barrier):
+    """CUDA-event time of each of `steps` steps, the L2 flushed (256 MiB write)
+    before every step; a barrier and a device synchronize on both sides."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        run()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def kernel_profile(q, torch, run, steps, flush, stream, barrier):
+    """A second pass of the same steps with the library's per-launch CUDA events on
+    (kept out of the headline pass): per-kernel launches, time and share, and the
+    launches per step."""
+    q.profile_enable(True)
+    time_steps(torch, run, steps, flush, stream, barrier)
+    prof, nlaunch = q.profile_read()
+    q.profile_enable(False)
+    by = {}
+    for kind, ms in prof:
+        d = by.setdefault(kind, [0, 0.0])
+        d[0] += 1
+        d[1] += ms
+    tot = sum(v[1] for v in by.values()) or 1.0
+    kernels = {k: {"launches": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / tot, 4)}
+               for k, v in sorted(by.items(), key=lambda kv: -kv[1][1])}
+    return kernels, by, nlaunch // max(1, steps)
+
+
+def pick_peak(P, clk):
+    """The bf16 denominator.  The burst figure applies to a timed region whose SM
+    clock stayed at its maximum; the fraction at the sampled clock and against the
+    sustained figure are reported beside it."""
+    sm = (clk or {}).get("sm_mhz")
+    smax = (clk or {}).get("sm_max_mhz") or P.get("sm_max_mhz")
+    return P["bf16"], (sm / smax if sm and smax else None)
+
+
+def gemm_roofline(wl, by, steps, P, clk):
+    g_ms = by.get("gemm_fwd", [0, 0.0])[1] + by.get("gemm_dx", [0, 0.0])[1]
+    g_n = by.get("gemm_fwd", [0, 0.0])[0] + by.get("gemm_dx", [0, 0.0])[0]
+    achieved = wl.gemm_flops * steps / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    peak, clk_ratio = pick_peak(P, clk)
+    return {"kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05 GEMM + LoRA K-steps; fwd and dX)",
+            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": (achieved / peak) if achieved else None,
+            "peak_source": f"{P['src']} bf16 burst (MEASURED_PEAKS.json: cuBLAS bf16, best of 10)",
+            "frac_vs_sustained": (achieved / P["bf16_sus"]) if achieved else None,
+            "frac_at_sampled_clock": (achieved / (peak * clk_ratio)) if achieved and clk_ratio else None,
+            "avg_launch_ms": g_ms / max(1, g_n), "launches_per_step": g_n // max(1, steps),
+            "flops_per_launch": wl.gemm_flops / max(1, g_n // max(1, steps)),
+            "traffic": traffic_for("qlora_gemm_kernel"),
+            "timing": "CUDA events around every GEMM launch, in a second timed pass of the same steps"}
+
+
+def e2e_measure(torch, wl, steps, stream, barrier, world, dev):
+    """The same step end to end through the public API: pinned host X and dY copied
+    to the device every step (the next step's inputs upload on their own stream into
+    the other of two device buffers while the current step computes, as a data
+    loader would) and the fp32 gradients read back; every copy lies inside the
+    timed region."""
+    import torch.distributed as dist
+    layers = wl.layers
+    flat = wl.bucket.flat
+    flat_host = torch.empty(flat.numel(), dtype=torch.float32).pin_memory()
+    h2d = sum(L["hX"].numel() * 2 + L["hdY"].numel() * 2 for L in layers)
+    d2h = flat_host.numel() * 4
+    xfer = torch.cuda.Stream(device=dev)
+    bufs = [[(L["X"], L["dY"]) for L in layers],
+            [(torch.empty_like(L["X"]), torch.empty_like(L["dY"])) for L in layers]]
+    uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def upload(b):
+        xfer.wait_event(consumed[b])
+        with torch.cuda.stream(xfer):
+            for (X, dY), L in zip(bufs[b], layers):
+                X.copy_(L["hX"], non_blocking=True)
+                dY.copy_(L["hdY"], non_blocking=True)
+        uploaded[b].record(xfer)
+
+    def step_on(b):
+        stream.wait_event(uploaded[b])
+        wl.run(bufs[b])
+        consumed[b].record(stream)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    xfer.wait_event(e0)
+    upload(0)
+    for i in range(steps):
+        if i + 1 < steps:
+            upload((i + 1) % 2)
+        step_on(i % 2)
+        flat_host.copy_(flat, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del bufs
+    return {"value": world * wl.flops * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "uploads": "next step's inputs overlap the current step (two buffers)"}
+
+
+def secondary_workload(q, torch, dev, name, steps, warmup, flush, stream, P):
+    """A further large-token workload at N = 1: median step, whole-step and GEMM
+    roofline fractions."""
+    wl = Workload(q, torch, dev, name, 0, pinned=False)
+    for _ in range(warmup):
+        wl.run()
+    torch.cuda.synchronize()
+    ms = time_steps(torch, wl.run, steps, flush, stream, lambda: None)
+    kernels, by, per_step = kernel_profile(q, torch, wl.run, steps, flush, stream, lambda: None)
+    med = statistics.median(ms)
+    roof = gemm_roofline(wl, by, steps, P, None)
+    out = {"workload": WORKLOAD_TEXT[name], "value": wl.flops / (med * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "ms_per_step": med, "ms_mean": statistics.mean(ms), "steps": steps,
+           "step_frac_of_peak": wl.flops / (med * 1e-3) / 1e12 / P["bf16"],
+           "gemm_achieved": roof["achieved"], "gemm_frac": roof["frac"],
+           "launches_per_step": per_step, "kernels": kernels}
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
+def small_layer(q, torch, dev, stream):
+    """The small single layer (16 tokens, W 1024x1024, r = 8): fwd+bwd in
+    microseconds, as separate calls (median of SMALL_CALLS, each bracketed by
+    events) and inside one CUDA graph of SMALL_CALLS back-to-back calls."""
+    wl = Workload(q, torch, dev, "small", 0, pinned=False)
+    for _ in range(5):
+        wl.run()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(SMALL_CALLS):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        wl.run()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    plain_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(SMALL_CALLS):
+            wl.run()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    a.record(cur)
+    g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    graph_us = 1e3 * a.elapsed_time(b) / SMALL_CALLS
+    del g, wl
+    return {"workload": WORKLOAD_TEXT["small"], "us_per_fwd_bwd": plain_us,
+            "us_per_fwd_bwd_in_graph": graph_us, "calls": SMALL_CALLS,
+            "TFLOP/s_in_graph": workload_flops("small") / (graph_us * 1e-6) / 1e12}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-subpaths", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the LLaMA-7B-shaped and small-layer measurements")
     ap.add_argument("--case", default=None,
-                    help="M,N,K: small profiling case (two fwd+bwd of one projection), no JSON")
+                    help="M,N,K[,r]: small profiling case (two fwd+bwd of one projection), no JSON")
     ap.add_argument("--quant-case", type=int, default=None,
                     help="N: profiling case, quantize + dequant of N heavy-tailed values twice, no JSON")
     args = ap.parse_args()
@@ -317,163 +590,57 @@ def main():
         if world > 1:
             dist.barrier()
 
-    hp = host_problems(rank)
     P = peaks()
     stream = torch.cuda.current_stream()
-
-    # ---- device-resident state (weights quantized once, like a model load)
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    from bit_nf4_quantized_19_b200.dp import GradBucket
-    layers = []
-    bucket = GradBucket([(N, K, RANK_R) for (_, N, K) in SHAPES], dev)
-    flat_grads = bucket.flat
-    flat_host = torch.empty(flat_grads.numel(), dtype=torch.float32).pin_memory()
-    for p, (dA, dB) in zip(hp, bucket.views):
-        M, N, K, r = p["M"], p["N"], p["K"], p["r"]
-        Wq = q.nf4_quantize(to_dev(p["W"]))
-        L = dict(M=M, N=N, K=K, r=r, s=p["s"], Wq=Wq, X=to_dev(p["X"]), dY=to_dev(p["dY"]),
-                 A=to_dev(p["A"]), B=to_dev(p["B"]),
-                 Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
-                 XA=torch.empty(M, r, dtype=torch.float32, device=dev),
-                 dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
-                 dA=dA, dB=dB, ws=q.make_workspace(M, N, K, r, dev))
-        L["hX"] = torch.from_numpy(np.ascontiguousarray(p["X"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        L["hdY"] = torch.from_numpy(np.ascontiguousarray(p["dY"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        layers.append(L)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    wl = Workload(q, torch, dev, HEADLINE, rank)
     torch.cuda.synchronize()
 
-    def step():
-        for L in layers:
-            q.linear_fwd(L["X"], L["Wq"], L["A"], L["B"], L["s"], workspace=L["ws"], Y=L["Y"],
-                         XA=L["XA"])
-            q.linear_bwd(L["dY"], L["X"], L["XA"], L["Wq"], L["A"], L["B"], L["s"],
-                         workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
-        bucket.allreduce_()       # the one exchange of data-parallel adapter training
-
-    flops_per_step_rank = sum(step_flops(M, N, K, RANK_R) for (M, N, K) in SHAPES)
-
     for _ in range(args.warmup):
-        step()
+        wl.run()
     torch.cuda.synchronize()
     code, flags = q.device_status()
     if code != 0:
         raise RuntimeError(f"device status {code} flags {flags} after warm-up")
 
-    # ---- timed region: K steps, L2 flushed before each, CUDA events per step
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    q.profile_enable(True)
+    # ---- headline timed region: K steps, L2 flushed before each, CUDA events per step,
+    # no library event recording inside it
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.fill_(float(i))
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-    prof, nlaunch = q.profile_read()
-    q.profile_enable(False)
-    barrier()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
+        step_ms = time_steps(torch, wl.run, args.steps, flush, stream, barrier)
+    med = statistics.median(step_ms)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([med], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        med = float(t.item())
     code, flags = q.device_status()
     if code != 0:
         raise RuntimeError(f"device status {code} flags {flags} after timing")
-    value = world * flops_per_step_rank * args.steps / (total_ms * 1e-3) / 1e12
+    value = world * wl.flops / (med * 1e-3) / 1e12
+    clocks = clk.summary()
 
-    # ---- per-kernel breakdown and the dominant kernel's roofline
-    by = {}
-    for kind, ms in prof:
-        d = by.setdefault(kind, [0, 0.0])
-        d[0] += 1
-        d[1] += ms
-    kern_total = sum(v[1] for v in by.values()) or 1.0
-    kernels = {k: {"launches": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / kern_total, 4)}
-               for k, v in sorted(by.items(), key=lambda kv: -kv[1][1])}
-    gemm_flops = args.steps * sum(2.0 * M * N * K + 2.0 * M * N * RANK_R + 2.0 * M * N * K
-                                  + 2.0 * M * K * RANK_R for (M, N, K) in SHAPES)
-    gemm_ms = by.get("gemm_fwd", [0, 0.0])[1] + by.get("gemm_dx", [0, 0.0])[1]
-    gemm_launches = by.get("gemm_fwd", [0, 0.0])[0] + by.get("gemm_dx", [0, 0.0])[0]
-    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
-    roof = {"kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05 GEMM + LoRA K-steps; fwd and dX)",
-            "bound": "tensor", "achieved": achieved, "peak": P["bf16_sus"], "unit": "TFLOP/s",
-            "frac": (achieved / P["bf16_sus"]) if achieved else None,
-            "peak_source": f"{P['src']} bf16 sustained (MEASURED_PEAKS.json)",
-            "avg_launch_ms": gemm_ms / max(1, gemm_launches),
-            "traffic": traffic_for("qlora_gemm_kernel")}
+    # ---- per-kernel breakdown and the dominant kernel's roofline (second pass)
+    kernels, by, launches_per_step = kernel_profile(q, torch, wl.run, args.steps, flush, stream, barrier)
+    roof = gemm_roofline(wl, by, args.steps, P, clocks)
+    roof["step_frac_of_peak"] = wl.flops / (med * 1e-3) / 1e12 / roof["peak"]
 
-    # ---- end to end through the public API: pinned host inputs -> device -> grads back.
-    # As a data loader would, the next step's inputs are uploaded (on their own stream,
-    # into the other of two device buffers) while the current step computes; every
-    # upload and every read-back of the gradients lies inside the timed region.
-    e2e_steps = max(3, min(args.steps, 30))
-    h2d = sum(L["hX"].numel() * 2 + L["hdY"].numel() * 2 for L in layers)
-    d2h = flat_host.numel() * 4
-    xfer = torch.cuda.Stream(device=dev)
-    bufs = [[(L["X"], L["dY"]) for L in layers],
-            [(torch.empty_like(L["X"]), torch.empty_like(L["dY"])) for L in layers]]
-    uploaded = [torch.cuda.Event(), torch.cuda.Event()]
-    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+    e2e = e2e_measure(torch, wl, max(3, min(args.steps, 10)), stream, barrier, world, dev)
+    del wl
+    torch.cuda.empty_cache()
 
-    def upload(b):
-        xfer.wait_event(consumed[b])          # the step that last read buffer b is done
-        with torch.cuda.stream(xfer):
-            for (X, dY), L in zip(bufs[b], layers):
-                X.copy_(L["hX"], non_blocking=True)
-                dY.copy_(L["hdY"], non_blocking=True)
-        uploaded[b].record(xfer)
-
-    def step_on(b):
-        stream.wait_event(uploaded[b])
-        for (X, dY), L in zip(bufs[b], layers):
-            q.linear_fwd(X, L["Wq"], L["A"], L["B"], L["s"], workspace=L["ws"], Y=L["Y"], XA=L["XA"])
-            q.linear_bwd(dY, X, L["XA"], L["Wq"], L["A"], L["B"], L["s"],
-                         workspace=L["ws"], dX=L["dX"], dA=L["dA"], dB=L["dB"])
-        bucket.allreduce_()
-        consumed[b].record(stream)
-
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    xfer.wait_event(e0)
-    upload(0)
-    for i in range(e2e_steps):
-        if i + 1 < e2e_steps:
-            upload((i + 1) % 2)
-        step_on(i % 2)
-        flat_host.copy_(flat_grads, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * flops_per_step_rank * e2e_steps / (e2e_ms * 1e-3) / 1e12,
-           "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "steps": e2e_steps, "uploads": "next step's inputs overlap the current step (two buffers)"}
-
-    # ---- HBM-bound subpaths (quantize / dequant of 1e9 values, skinny forward): single-GPU
-    # measurements, taken at N = 1 only so a multi-GPU run stays short and symmetric
-    subpaths = None
+    # ---- single-GPU extras at N = 1 only, so a multi-GPU run stays short and symmetric
+    others, subpaths = None, None
+    if world == 1 and not args.no_secondary:
+        others = {"llama7b": secondary_workload(q, torch, dev, "llama7b", args.steps, args.warmup,
+                                                flush, stream, P),
+                  "small": small_layer(q, torch, dev, stream)}
     if not args.no_subpaths and world == 1:
         subpaths = hbm_subpaths(q, torch, dev, stream, P, flush)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        hp0 = host_problems(0)
-        tokens, wrows = 512, 2048
-        fl, sec = oracle_sample(hp0, tokens, wrows)
+        tokens, wrows = CPU_SAMPLE[HEADLINE]
+        fl, sec = oracle_sample(sample_problems(HEADLINE, tokens, wrows), tokens, wrows)
         cores, blas = cpu_info()
         cpu_baseline = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": blas or cores,
                         "kind": "oracle",
@@ -483,32 +650,36 @@ def main():
     if world > 1:
         dist.barrier()
     if rank == 0:
+        wld = WORKLOADS[HEADLINE]
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": med,
+                "ms_per_step_mean": statistics.mean(step_ms),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic (seeded): W ~ N(0,0.02) bf16 quantized to NF4, X, dY ~ N(0,1), "
+                "data": "synthetic (seeded): W ~ N(0,0.015) bf16 quantized to NF4, X, dY ~ N(0,1), "
                         "A ~ N(0,1/r), B ~ N(0,0.01)",
-                "config": {"workload": WORKLOAD, "global_batch": 4096 * world,
-                           "tokens_per_gpu": 4096, "parallelism": f"dp{world}",
+                "config": {"workload": WORKLOAD, "global_batch": wld["shapes"][0][0] * world,
+                           "tokens_per_gpu": wld["shapes"][0][0], "lora_r": wld["r"],
+                           "lora_alpha": wld["alpha"], "parallelism": f"dp{world}",
                            "l2": "flushed (256 MiB write) before every timed step",
-                           "flops_per_step_per_gpu": flops_per_step_rank},
+                           "step_time": "median of the timed steps",
+                           "flops_per_step_per_gpu": workload_flops(HEADLINE)},
                 "roofline": roof, "cpu_baseline": cpu_baseline, "e2e": e2e,
-                "gpu_launches": nlaunch, "clocks": clk.summary(), "kernels": kernels,
-                "subpaths": subpaths}
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "kernels": kernels,
+                "other_workloads": others, "subpaths": subpaths}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
 
 
-def profile_case(M, N, K, r=RANK_R):
+def profile_case(M, N, K, r=16):
     """Two forward + backward passes of one projection through the public API
     (seeded device inputs); the case that the ncu captures under profiles/ use."""
     import torch
     import bit_nf4_quantized_19_b200 as q
     g = torch.Generator(device="cuda")
     g.manual_seed(0)
-    W = (torch.randn(N, K, generator=g, device="cuda") * W_STD).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
     X = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
     dY = torch.randn(M, N, generator=g, device="cuda").to(torch.bfloat16)
     A = (torch.randn(K, r, generator=g, device="cuda") / r).to(torch.bfloat16)
@@ -516,8 +687,8 @@ def profile_case(M, N, K, r=RANK_R):
     Wq = q.nf4_quantize(W)
     ws = q.make_workspace(M, N, K, r, X.device)
     for _ in range(2):
-        Y, XA = q.linear_fwd(X, Wq, A, B, ALPHA / r, workspace=ws)
-        q.linear_bwd(dY, X, XA, Wq, A, B, ALPHA / r, workspace=ws)
+        Y, XA = q.linear_fwd(X, Wq, A, B, 2.0, workspace=ws)
+        q.linear_bwd(dY, X, XA, Wq, A, B, 2.0, workspace=ws)
     torch.cuda.synchronize()
     code, flags = q.device_status()
     print("case", M, N, K, "status", code, flags)
@@ -582,7 +753,7 @@ def hbm_subpaths(q, torch, dev, stream, P, flush):
     gen = torch.Generator(device=dev)
     gen.manual_seed(1)
     for (M, N, K) in SKINNY:
-        r = RANK_R
+        r = 16
         Wb = (torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
         Wq = q.nf4_quantize(Wb)
         X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
@@ -611,7 +782,7 @@ def hbm_subpaths(q, torch, dev, stream, P, flush):
     # together exceeds 2.5x the L2, called back to back as the consecutive layers of
     # a decode step are, so every call streams its weight from HBM
     for (N, K) in sorted({(n, k) for _, n, k in SKINNY}):
-        r = RANK_R
+        r = 16
         Wb = (torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
         Wq0 = q.nf4_quantize(Wb)
         L = max(8, -(-GRAPH_STREAM_BYTES // Wq0.nbytes))

@@ -71,7 +71,7 @@ SIGNATURES = {
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "prep", "project", "gemm_fwd", "gemm_dx",
-                "grad", "unused", "skinny"]
+                "grad", "skinny"]
 PROFILE_CAP = 4096
 
 _LIB = None

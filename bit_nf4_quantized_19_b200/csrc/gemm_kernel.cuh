@@ -18,9 +18,12 @@
 //   warp 0        TMA producer of the activation tiles (X / dY, or the LoRA
 //                 hi/lo operand).
 //   warp 1        TMEM allocator and single-thread MMA issuer.
-//   warp 2        TMA producer of the packed 4-bit weight tiles + block
-//                 constants (its own ring, so the small weight stream runs
-//                 ahead of the activation ring instead of waiting behind it).
+//   warp 2        weight producer: lane 0 TMA-loads the packed 4-bit codes of
+//                 each stage into their own ring (so the small weight stream runs
+//                 ahead of the activation ring instead of waiting behind it); all
+//                 32 lanes rebuild the stage's 128 block constants
+//                 RN32(q8 * step) from the 8-bit codes and the fp32 group
+//                 constants (read one stage ahead) next to them.
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
 //   warps 8..15   dequant producers, two warpgroups taking alternate stages:
 //                 packed codes + block constant -> bf16 tile in the
@@ -31,12 +34,15 @@
 //
 // Last-wave split: with T tiles on G persistent CTAs, T mod G tiles are left for a
 // last round in which most SMs would idle.  When at most G/2 remain, each of them
-// is split along the contraction into two halves taken by CTAs 2i and 2i+1: the
-// first half writes its fp32 partial tile to scratch and publishes it under a
-// per-launch epoch (release); the second half runs the rest of the contraction and
-// the LoRA steps, waits for the epoch (acquire, bounded), and adds the partial in
-// its epilogue.  The first half never waits, and the grid has at most one CTA per
-// SM, so the wait always ends.
+// is split along the contraction into two halves taken by CTAs 2i and 2i+1 (the
+// second half also runs the LoRA steps).  Whichever half finishes first stores its
+// fp32 partial tile to scratch and publishes it; the other adds that partial to its
+// own accumulator and writes the output (last arriver).  A half learns its role
+// from an atomic arrival counter per split tile, which a kernel earlier in the same
+// call sets to zero.  The only wait is the last arriver's, for a partial whose
+// writer has already arrived (so is running), which makes it independent of how
+// the CTAs are scheduled.  The sum of two fp32 values does not depend on their
+// order, so the result is the same whichever half finishes first.
 #pragma once
 #include "common.cuh"
 
@@ -61,6 +67,8 @@ constexpr int kBStageBytes = kBN * 128;   // 32 KB
 constexpr int kAStageBytes = kWT * 128;   // 16 KB
 constexpr int kWStageBytes = 4096;        // packed codes of one stage
 constexpr int kSStageBytes = 512;         // 128 fp32 block constants of one stage
+constexpr uint32_t kSplitArrive = 1u;     // split-tile counter: one per arriving half
+constexpr uint32_t kSplitReady = 16u;     // added once the first half's partial is stored
 constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
 
 constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStagesB * kBStageBytes +
@@ -80,15 +88,17 @@ struct GemmParams {
   int kb_lora;       // LoRA stages: ceil(2r / 64)
   int r;
   int lora_ld;       // row pitch of the LoRA weight operand source: N (B [r,N]) or r (A [K,r])
+  int KB;            // 64-value blocks per weight row: K / 64
+  const uint8_t *q8;       // 8-bit block constants of W, [N * KB]
+  const float *step;       // fp32 group constants, one per 256 blocks
   const uint16_t *lora_w;  // fwd: B [r, N];  dX: A [K, r]
   uint16_t *out;     // Y [M, N] or dX [M, K]
   uint64_t limit_ns;
   int split_base;    // first tile of the split last round (a multiple of the grid size)
   int split_count;   // tiles split into two contraction halves (0: no split)
   int kb_mid;        // first main stage of the second half
-  float *scratch;    // [split_count][128][256] fp32 partial tiles of the first halves
-  unsigned long long *flags;   // [split_count]: epoch once the partial tile is complete
-  unsigned long long epoch;    // unique per launch
+  float *scratch;    // [split_count][128][256] fp32 partial tile of the half that finishes first
+  unsigned int *flags;   // [split_count] arrival counters, zero at launch
   float levels[16];
 };
 
@@ -117,13 +127,34 @@ QDEV bool gemm_item(const GemmParams &p, int num_tiles, int it, GemmItem &w) {
   return true;
 }
 
-QDEV unsigned long long ld_acquire_u64(const unsigned long long *a) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+QDEV uint32_t ld_acquire_u32(const unsigned int *a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
   return v;
 }
-QDEV void st_release_u64(unsigned long long *a, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(v) : "memory");
+QDEV void red_release_add_u32(unsigned int *a, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+QDEV uint32_t atom_acq_rel_add_u32(unsigned int *a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+  return old;
+}
+
+// The 128 block constants of one weight stage, RN32(q8 * step) for stage slot idx =
+// lane + 32 i:  fwd: weight row w0 + idx, block kb;  dX: weight row kb*64 + (idx & 63),
+// block w0/64 + (idx >> 6).  Raw values are loaded here and multiplied when stored.
+template <int MODE>
+QDEV void load_stage_scales(const GemmParams &p, int w0, int kb, int lane, uint32_t (&q)[4], float (&st)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = lane + 32 * i;
+    int64_t b;
+    if (MODE == kModeFwd) b = static_cast<int64_t>(w0 + idx) * p.KB + kb;
+    else b = static_cast<int64_t>(kb * kBK + (idx & 63)) * p.KB + (w0 >> 6) + (idx >> 6);
+    q[i] = __ldg(p.q8 + b);
+    st[i] = __ldg(p.step + (b >> 8));
+  }
 }
 QDEV void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -131,7 +162,6 @@ template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,   // X or dY, bf16 [M, contraction]
                       const __grid_constant__ CUtensorMap tm_codes, // packed codes, u8 [N, K/2]
-                      const __grid_constant__ CUtensorMap tm_scale, // block constants, f32 [K/64, N]
                       const __grid_constant__ CUtensorMap tm_lora,  // hi/lo LoRA operand, bf16 [M, 2r]
                       const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -153,6 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   float *sL = reinterpret_cast<float *>(abort_flag + 1);
+  volatile int *split_role = reinterpret_cast<volatile int *>(sL + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -164,7 +195,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full_A[i], 4);
       mbar_init(&empty_A[i], 1);
     }
-    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 1); mbar_init(&empty_W[i], 4); }
+    // full_W: the TMA's expect_tx arrival plus one per lane of the weight producer
+    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 33); mbar_init(&empty_W[i], 4); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -174,7 +206,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_act);
     prefetch_tmap(&tm_codes);
-    prefetch_tmap(&tm_scale);
     prefetch_tmap(&tm_lora);
   }
   if (warp == 1) {
@@ -220,32 +251,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ weight producer
-    if (lane == 0) {
-      int ws = 0;
-      uint32_t wph = 0;
-      uint32_t armedW = 0, lastW = 0;
-      bool ok = true;
-      GemmItem w;
-      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
-        const int w0 = (w.tile % p.num_w_tiles) * kWT;
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!wait_bar(&empty_W[ws], wph ^ 1u, wt)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_W[ws], kWStageBytes + kSStageBytes);
-          if (MODE == kModeFwd) {
-            // codes: 32 bytes (64 values of K) x 128 weight rows; constants S[kb][w0 .. w0+128)
-            tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
-            tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], w0, kb);
-          } else {
-            // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..;
-            // constants S[w0/64 + {0,1}][kb*64 .. kb*64+64)
-            tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
-            tma_load_2d(sS + ws * 128, &tm_scale, &full_W[ws], kb * kBK, w0 / kBK);
-          }
-          armedW |= 1u << ws;
-          lastW = (lastW & ~(1u << ws)) | (wph << ws);
-          if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
-        }
+    int ws = 0;
+    uint32_t wph = 0;
+    uint32_t armedW = 0, lastW = 0;
+    GemmItem w;
+    int it = 0;
+    bool have = gemm_item(p, num_tiles, 0, w);
+    int kb = have ? w.kb0 : 0;
+    uint32_t q_cur[4] = {0u, 0u, 0u, 0u};
+    float s_cur[4] = {0.f, 0.f, 0.f, 0.f};
+    if (have) load_stage_scales<MODE>(p, (w.tile % p.num_w_tiles) * kWT, kb, lane, q_cur, s_cur);
+    while (have) {
+      const int w0 = (w.tile % p.num_w_tiles) * kWT;
+      // the next stage's raw constants are requested now and used one iteration later
+      GemmItem wn = w;
+      int itn = it, kbn = kb + 1;
+      bool have_n = true;
+      if (kbn >= w.kb1) {
+        itn = it + 1;
+        have_n = gemm_item(p, num_tiles, itn, wn);
+        kbn = have_n ? wn.kb0 : 0;
       }
+      uint32_t q_nxt[4] = {0u, 0u, 0u, 0u};
+      float s_nxt[4] = {0.f, 0.f, 0.f, 0.f};
+      if (have_n) load_stage_scales<MODE>(p, (wn.tile % p.num_w_tiles) * kWT, kbn, lane, q_nxt, s_nxt);
+      // warp-uniform: every lane arrives on full_W below
+      if (!__all_sync(0xffffffffu, wait_bar(&empty_W[ws], wph ^ 1u, wt))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full_W[ws], kWStageBytes);
+        if (MODE == kModeFwd) {
+          // codes: 32 bytes (64 values of K) x 128 weight rows
+          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
+        } else {
+          // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..
+          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
+        }
+        armedW |= 1u << ws;
+        lastW = (lastW & ~(1u << ws)) | (wph << ws);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        sS[ws * 128 + lane + 32 * i] = __fmul_rn(static_cast<float>(q_cur[i]), s_cur[i]);
+      mbar_arrive(&full_W[ws]);
+      if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
+      w = wn;
+      it = itn;
+      kb = kbn;
+      have = have_n;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { q_cur[i] = q_nxt[i]; s_cur[i] = s_nxt[i]; }
+    }
+    if (lane == 0) {
       volatile int no_abort = 0;
       const Waiter final_wt{&no_abort, p.limit_ns};
       for (int s = 0; s < kStagesW; ++s)
@@ -324,20 +380,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int sidx = w.tile - p.split_base;                  // split tiles only
       float *prow = (w.part != 0) ? p.scratch + (static_cast<int64_t>(sidx) * kWT + row) * kBN : nullptr;
-      if (w.part == 2) {
-        // the first half's partial tile: one thread waits for its epoch (bounded)
+      // role: 0 a whole tile; 1 the first half of a split tile to finish (stores its
+      // partial); 2 the second (adds the partial and writes the output)
+      int role = 0;
+      if (w.part != 0) {
         if (warp == 4 && lane == 0) {
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u64(p.flags + sidx) != p.epoch) {
-            if (*reinterpret_cast<volatile int *>(abort_flag) || globaltimer_ns() - t0 > p.limit_ns) {
-              *reinterpret_cast<volatile int *>(abort_flag) = 1;
-              atomicOr(&g_device_status, kStatTimeout);
-              break;
+          const uint32_t old = atom_acq_rel_add_u32(p.flags + sidx, kSplitArrive);
+          const int rl = ((old & (kSplitReady - 1u)) == 0u) ? 1 : 2;
+          if (rl == 2) {
+            // the other half has arrived, so it is running: wait (bounded) for its partial
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_u32(p.flags + sidx) < kSplitReady) {
+              if (*reinterpret_cast<volatile int *>(abort_flag) || globaltimer_ns() - t0 > p.limit_ns) {
+                *reinterpret_cast<volatile int *>(abort_flag) = 1;
+                atomicOr(&g_device_status, kStatTimeout);
+                break;
+              }
             }
           }
+          *split_role = rl;
         }
         epilogue_bar();
-        __threadfence();
+        role = *split_role;
+        if (role == 2) __threadfence();
       }
       uint16_t *outc = p.out + w0 + row;
       for (int cc = 0; cc < kBN / 32; ++cc) {
@@ -346,7 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                static_cast<uint32_t>(acc * kBN + cc * 32),
                            v);
         tmem_wait_ld();
-        if (w.part == 1) {
+        if (role == 1) {
           float4 *d4 = reinterpret_cast<float4 *>(prow + cc * 32);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -354,7 +419,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           continue;
         }
-        if (w.part == 2) {
+        if (role == 2) {
           const float4 *s4 = reinterpret_cast<const float4 *>(prow + cc * 32);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -375,11 +440,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (w.part == 1) {
+      if (role == 1) {
         // publish the partial tile: every epilogue thread's stores, then one release
         __threadfence();
         epilogue_bar();
-        if (warp == 4 && lane == 0) st_release_u64(p.flags + sidx, p.epoch);
+        if (warp == 4 && lane == 0) red_release_add_u32(p.flags + sidx, kSplitReady);
       }
       tc_fence_before();
       __syncwarp();

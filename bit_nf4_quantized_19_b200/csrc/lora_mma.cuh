@@ -54,6 +54,10 @@ struct LoraMmaParams {
   int rows1;
   float *out1;
   int layout1;
+  // Words that a later kernel of the same call expects to find zero (the fused GEMM's
+  // split-tile arrival counters); CTA (0, 0) clears them.  May be null.
+  unsigned int *zero;
+  int zero_n;
 };
 
 constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of a tile
@@ -93,6 +97,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.zero && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = tid; i < p.zero_n; i += kLmThreads) p.zero[i] = 0u;
   const bool second = static_cast<int>(blockIdx.x) >= p.tiles0;
   const int row0 = (static_cast<int>(blockIdx.x) - (second ? p.tiles0 : 0)) * kLmRows;
   const int rows = second ? p.rows1 : p.rows;

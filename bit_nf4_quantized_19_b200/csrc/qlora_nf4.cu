@@ -3,8 +3,6 @@
 #include "qlora_nf4.h"
 
 #include <atomic>
-#include <chrono>
-#include <random>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -46,22 +44,6 @@ struct DeviceInfo {
   int sms = 0;
   int major = 0;
   bool gemm_attr_set = false;
-  // A second stream of the library's own, for work that only depends on the weight
-  // (the block-constant expansion) to run beside the rank-r projection.  fork_mu
-  // keeps each fork / join pair of event records and waits together.
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-  std::mutex fork_mu;
-};
-// Joins the side stream back into the caller's stream when a forked call leaves
-// early on an error, so no side-stream work outlives the call's ordering.
-struct ForkGuard {
-  DeviceInfo *d;
-  cudaStream_t st;
-  bool pending = false;
-  ~ForkGuard() {
-    if (pending) cudaStreamWaitEvent(st, d->ev_join, 0);
-  }
 };
 
 constexpr int kMaxDevices = 64;
@@ -81,12 +63,6 @@ qlora_status device_info(DeviceInfo **out) {
       return QLORA_ERR_CUDA;
     d.sms = sms;
     d.major = major;
-    if (cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&d.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&d.ev_join, cudaEventDisableTiming) != cudaSuccess) {
-      d.sms = 0;
-      return QLORA_ERR_CUDA;
-    }
   }
   if (d.major != 10) return QLORA_ERR_NO_DEVICE;
   if (!d.gemm_attr_set) {
@@ -301,7 +277,7 @@ int64_t pad8(int64_t m) { return (m + 7) / 8 * 8; }
 struct GemmSplit {
   int base = 0, count = 0;
   size_t scratch_bytes() const { return static_cast<size_t>(count) * kWT * kBN * 4; }
-  size_t flag_bytes() const { return static_cast<size_t>(count) * 8; }
+  size_t flag_bytes() const { return static_cast<size_t>(count) * 4; }
 };
 GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, int sms) {
   GemmSplit g;
@@ -317,18 +293,17 @@ GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, int sms) {
 }
 size_t split_workspace(const GemmSplit &g) { return align256(g.scratch_bytes()) + align256(g.flag_bytes()); }
 
-// A value no flag left in a reused workspace can hold by chance: a per-process
-// random high half and a per-launch counter.
-unsigned long long next_epoch() {
-  static std::atomic<unsigned long long> ctr{
-      (static_cast<unsigned long long>(std::random_device{}()) << 32) |
-      static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count() & 0xFFFF0000ull)};
-  return ctr.fetch_add(1) + 1;
-}
+// Scratch of one split GEMM launch, carved from the workspace before the call's first
+// launch: its arrival counters are cleared by the rank-r projection that precedes the
+// GEMM in the same call.
+struct SplitScratch {
+  GemmSplit g;
+  float *partial = nullptr;
+  unsigned int *flags = nullptr;
+};
 
 size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
-  b += align256(static_cast<size_t>(N) * (K / 64) * 4);        // expanded block constants
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*XA hi/lo
   b += align256(static_cast<size_t>(M) * r * 4);               // XA when XA_out is NULL
@@ -338,7 +313,6 @@ size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
 
 size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t b = 0;
-  b += align256(static_cast<size_t>(N) * (K / 64) * 4);
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T (XA recompute)
   b += align256(static_cast<size_t>(M) * r * 4);               // G
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*G hi/lo
@@ -347,6 +321,14 @@ size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   b += align256(static_cast<size_t>(M) * r * 4);               // XA recomputed
   b += split_workspace(gemm_split(M, K, N, sms));              // last-wave partial tiles (dX)
   return b + 256;
+}
+
+bool take_split(Workspace &ws, const GemmSplit &g, SplitScratch &out) {
+  out.g = g;
+  if (!g.count) return true;
+  out.partial = static_cast<float *>(ws.take(g.scratch_bytes()));
+  out.flags = static_cast<unsigned int *>(ws.take(g.flag_bytes()));
+  return out.partial && out.flags;
 }
 
 qlora_status check_nf4(const qlora_nf4_t *Wq) {
@@ -362,16 +344,6 @@ qlora_status check_linear_shape(int64_t M, const qlora_nf4_t *Wq, int r) {
   if (Wq->rows % 128 != 0 || Wq->cols % 128 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (Wq->rows > (1ll << 24) || Wq->cols > (1ll << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   return QLORA_OK;
-}
-
-qlora_status launch_expand_scales(const qlora_nf4_t *Wq, float *S, cudaStream_t st, int sms) {
-  const int N = static_cast<int>(Wq->rows), KB = static_cast<int>(Wq->cols / 64);
-  const int64_t total = static_cast<int64_t>(N) * KB;
-  int grid = static_cast<int>((total + 255) / 256);
-  if (grid > sms * 8) grid = sms * 8;
-  LaunchTimer lt(QLORA_K_EXPAND, st);
-  nf4_expand_scales_kernel<<<grid, 256, 0, st>>>(Wq->q8, Wq->step, N, KB, S);
-  return cuda_status(cudaGetLastError());
 }
 
 int grid_for(int64_t total, int sms) {
@@ -452,8 +424,12 @@ qlora_status launch_lora_mma(const LmOperands &o, int64_t contraction, int nn, L
 // XA = X A (or G = dY B^T): fp32 [M, r] plus hi/lo of s*result in [M, 2r] and/or [2r, pad8(M)].
 qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const uint16_t *qT,
                                int r, float s, float *out, uint16_t *hl, uint16_t *hlT, int sms,
-                               cudaStream_t st) {
+                               cudaStream_t st, const SplitScratch *clear = nullptr) {
   LoraMmaParams p{};
+  if (clear && clear->g.count) {
+    p.zero = clear->flags;
+    p.zero_n = clear->g.count;
+  }
   p.grad = 0;
   p.r = r;
   p.s = s;
@@ -467,7 +443,7 @@ qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const 
 
 qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *hlT, int sms,
                            cudaStream_t st) {
-  LaunchTimer lt(QLORA_K_EXPAND, st);
+  LaunchTimer lt(QLORA_K_PREP, st);
   hilo_t_kernel<<<grid_for(M * r, sms), 256, 0, st>>>(v, static_cast<int>(M), r, s, hlT,
                                                        static_cast<int>(pad8(M)));
   return cuda_status(cudaGetLastError());
@@ -492,7 +468,7 @@ qlora_status launch_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int6
 }
 
 qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT, int sms, cudaStream_t st) {
-  LaunchTimer lt(QLORA_K_EXPAND, st);
+  LaunchTimer lt(QLORA_K_PREP, st);
   transpose_bf16_kernel<<<grid_for(K * r, sms), 256, 0, st>>>(A, static_cast<int>(K), r, AT);
   return cuda_status(cudaGetLastError());
 }
@@ -619,26 +595,23 @@ qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, 
 }
 
 // One fused GEMM launch.  MODE fwd: Y = X deq(W)^T + LoRA; MODE dx: dX = dY deq(W) + LoRA.
+// `sp` is the launch's split scratch, its counters already cleared in stream order.
 template <int MODE>
-qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, const float *S,
+qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
                          const uint16_t *lora_act_hl, const uint16_t *lora_w, int r,
-                         uint16_t *out, Workspace &ws, int sms, cudaStream_t st) {
+                         uint16_t *out, const SplitScratch &sp, int sms, cudaStream_t st) {
   const int64_t N = Wq->rows, K = Wq->cols;
   const int64_t contraction = (MODE == kModeFwd) ? K : N;
-  CUtensorMap tm_act, tm_codes, tm_scale, tm_lora;
+  CUtensorMap tm_act, tm_codes, tm_lora;
   if (!make_map_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, contraction, M, contraction * 2,
                    kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
   if (MODE == kModeFwd) {
     if (!make_map_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, 32, kWT,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&tm_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S, N, K / 64, N * 4, kWT, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return QLORA_ERR_CUDA;
   } else {
     if (!make_map_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&tm_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S, N, K / 64, N * 4, 64, 2,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return QLORA_ERR_CUDA;
   }
@@ -655,6 +628,9 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, 
   p.kb_lora = (2 * r + kBK - 1) / kBK;
   p.r = r;
   p.lora_ld = (MODE == kModeFwd) ? static_cast<int>(N) : r;
+  p.KB = static_cast<int>(K / 64);
+  p.q8 = Wq->q8;
+  p.step = Wq->step;
   p.lora_w = lora_w;
   p.out = out;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
@@ -662,19 +638,15 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq, 
   std::memcpy(p.levels, T.levels, sizeof(p.levels));
   const int tiles = p.num_m_tiles * p.num_w_tiles;
   const int grid = tiles < sms ? tiles : sms;
-  const GemmSplit sp = gemm_split(M, (MODE == kModeFwd) ? N : K, contraction, sms);
-  p.split_base = sp.base;
-  p.split_count = sp.count;
+  const GemmSplit g = gemm_split(M, (MODE == kModeFwd) ? N : K, contraction, sms);
+  if (g.count != sp.g.count || g.base != sp.g.base) return QLORA_ERR_WORKSPACE;
+  p.split_base = g.base;
+  p.split_count = g.count;
   p.kb_mid = p.kb_main / 2;
-  if (sp.count) {
-    p.scratch = static_cast<float *>(ws.take(sp.scratch_bytes()));
-    p.flags = static_cast<unsigned long long *>(ws.take(sp.flag_bytes()));
-    if (!p.scratch || !p.flags) return QLORA_ERR_WORKSPACE;
-    p.epoch = next_epoch();
-  }
+  p.scratch = sp.partial;
+  p.flags = sp.flags;
   LaunchTimer lt(MODE == kModeFwd ? QLORA_K_GEMM_FWD : QLORA_K_GEMM_DX, st);
-  qlora_gemm_kernel<MODE><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_scale,
-                                                                      tm_lora, p);
+  qlora_gemm_kernel<MODE><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_lora, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -808,30 +780,17 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
     }
   }
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
-  float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
   uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  if (!S || !AT || !hl || !xa) return QLORA_ERR_WORKSPACE;
-  // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps
-  {
-    // the block constants depend only on the weight: expand them on the side stream
-    // while X*A runs here, and join before the GEMM
-    std::lock_guard<std::mutex> lk(d->fork_mu);
-    if (cudaEventRecord(d->ev_fork, stream) != cudaSuccess ||
-        cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    ForkGuard fg{d, stream};
-    if ((st = launch_expand_scales(Wq, S, d->side, d->sms)) != QLORA_OK) return st;
-    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess) return QLORA_ERR_CUDA;
-    fg.pending = true;
-    if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-    if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream)) != QLORA_OK)
-      return st;
-    fg.pending = false;
-    if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
-  }
-  return launch_gemm<kModeFwd>(X, M, Wq, S, hl, B, r, Y, ws, d->sms, stream);
+  SplitScratch sp;
+  if (!AT || !hl || !xa || !take_split(ws, gemm_split(M, N, K, d->sms), sp)) return QLORA_ERR_WORKSPACE;
+  // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps;
+  // the projection also clears the GEMM's split counters
+  if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream, &sp)) != QLORA_OK)
+    return st;
+  return launch_gemm<kModeFwd>(X, M, Wq, hl, B, r, Y, sp, d->sms, stream);
 }
 
 qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
@@ -853,27 +812,15 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
   if (!workspace || workspace_bytes < bwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   const size_t hlT_bytes = static_cast<size_t>(2 * r) * pad8(M) * 2;
-  float *S = static_cast<float *>(ws.take(static_cast<size_t>(N) * (K / 64) * 4));
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
   float *G = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   uint16_t *ghl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   uint16_t *ghlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
   float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  if (!S || !AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
-  std::unique_lock<std::mutex> lk(d->fork_mu, std::defer_lock);
-  ForkGuard fg{d, stream};
-  if (dX) {
-    // the block constants depend only on the weight: expand them on the side stream
-    // while the rank-r products below run here, and join before the dX GEMM
-    lk.lock();
-    if (cudaEventRecord(d->ev_fork, stream) != cudaSuccess ||
-        cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    if ((st = launch_expand_scales(Wq, S, d->side, d->sms)) != QLORA_OK) return st;
-    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess) return QLORA_ERR_CUDA;
-    fg.pending = true;
-  }
+  SplitScratch sp;
+  if (!AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
+  if (dX && !take_split(ws, gemm_split(M, K, N, d->sms), sp)) return QLORA_ERR_WORKSPACE;
   // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from X and A)
   if (XA) {
     if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
@@ -882,13 +829,11 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
     if ((st = launch_projection(X, M, K, AT, r, s, xa_ws, nullptr, xahlT, d->sms, stream)) != QLORA_OK)
       return st;
   }
-  // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA)
-  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream)) != QLORA_OK) return st;
+  // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA); clears the dX GEMM's
+  // split counters
+  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream, &sp)) != QLORA_OK) return st;
   if (dX) {
-    fg.pending = false;
-    if (cudaStreamWaitEvent(stream, d->ev_join, 0) != cudaSuccess) return QLORA_ERR_CUDA;
-    lk.unlock();
-    if ((st = launch_gemm<kModeDx>(dY, M, Wq, S, ghl, A, r, dX, ws, d->sms, stream)) != QLORA_OK) return st;
+    if ((st = launch_gemm<kModeDx>(dY, M, Wq, ghl, A, r, dX, sp, d->sms, stream)) != QLORA_OK) return st;
   }
   // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
   return launch_grads(X, dY, M, K, N, ghlT, xahlT, r, dA, dB, d->sms, stream);

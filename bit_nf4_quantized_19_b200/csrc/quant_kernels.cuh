@@ -341,19 +341,4 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
   }
 }
 
-// Per-block constants expanded for the fused GEMM, stored transposed:
-// S[kb][n] = RN32(q8[n*KB + kb] * step[(n*KB + kb) / 256]),  KB = K / 64.
-__global__ void __launch_bounds__(256) nf4_expand_scales_kernel(
-    const uint8_t *__restrict__ q8, const float *__restrict__ step, int N, int KB,
-    float *__restrict__ S) {
-  const int64_t total = static_cast<int64_t>(N) * KB;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int kb = static_cast<int>(i / N);
-    const int nrow = static_cast<int>(i - static_cast<int64_t>(kb) * N);
-    const int64_t b = static_cast<int64_t>(nrow) * KB + kb;
-    S[i] = __fmul_rn(static_cast<float>(q8[b]), step[b >> 8]);
-  }
-}
-
 }  // namespace qlora

@@ -26,7 +26,10 @@
  *     qlora_get_device_status() reads and clears.
  *   - Weight layout: W is [N, K] (out x in, the nn.Linear layout), flattened
  *     row-major for quantization.  X [M, K], Y [M, N], A [K, r], B [r, N].
- *   - Results are deterministic: no atomics, fixed reduction order.
+ *   - Results are deterministic: every reduction runs in a fixed order.  The one
+ *     atomic, the arrival counter of a GEMM tile split in two contraction halves,
+ *     only decides which half adds the other's partial sum, and a sum of two
+ *     fp32 values does not depend on their order.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -140,12 +143,13 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * Shapes: M >= 1; N % 128 == 0; K % 128 == 0; r % 8 == 0, 8 <= r <= 128.
  * Execution: with M <= 16 tokens (and a contraction short enough for its
  * shared-memory plan) the call takes the few-token path: X A in one small
- * launch and the weight pass as its programmatic dependent.  Otherwise the
- * block-constant expansion runs on a stream the library owns, forked from
- * `stream` by an event record and joined back by an event wait before the
- * GEMM.  Either way all work is ordered after what `stream` already holds and
- * before what is enqueued to `stream` later, and the call can be captured into
- * a CUDA graph.
+ * launch and the weight pass as its programmatic dependent.  Otherwise it
+ * launches, in order on `stream`, the transpose of A, the rank-r projection
+ * X A (which also clears the GEMM's split counters in the workspace) and the
+ * fused dequant GEMM, which rebuilds the block constants RN32(q8 * step) on
+ * chip.  All work is ordered after what `stream` already holds and before what
+ * is enqueued to `stream` later; no other stream is used, and the call can be
+ * captured into a CUDA graph and replayed with new inputs in the same buffers.
  */
 qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
                               const uint16_t *A, const uint16_t *B, int r, float s,
@@ -184,8 +188,7 @@ qlora_status qlora_linear_fwd_noalloc(const uint16_t *X, int64_t M, const qlora_
 /*
  * Backward of the adapted linear layer ([STEPS] Step 6: gradients flow through
  * the dequantized weights into the adapters; W is frozen, no dW).  Ordering and
- * graph capture as qlora_linear_fwd (the block-constant expansion for dX runs on
- * the library's stream between a fork and a join on `stream`):
+ * graph capture as qlora_linear_fwd (everything runs on `stream`):
  *   G  = dY B^T                   (fp32 [M, r], internal)
  *   dX = dY deq(W) + s * G A^T    (bf16 [M, K]; skipped when dX is NULL)
  *   dA = s * X^T G                (fp32 [K, r])
@@ -232,16 +235,14 @@ uint32_t qlora_set_wait_limit_us(uint32_t limit_us);
 typedef enum {
   QLORA_K_QUANTIZE = 0,     /* nf4 quantize + double quant          */
   QLORA_K_DEQUANT = 1,      /* standalone dequant                   */
-  QLORA_K_EXPAND = 2,       /* operand preparation: block-constant  */
-                            /* expansion, A^T, hi/lo of a saved XA  */
+  QLORA_K_PREP = 2,         /* operand preparation: A^T, hi/lo of a */
+                            /* saved XA                             */
   QLORA_K_PROJECT = 3,      /* XA = X A or G = dY B^T (+ hi/lo)     */
   QLORA_K_GEMM_FWD = 4,     /* fused dequant GEMM, forward          */
   QLORA_K_GEMM_DX = 5,      /* fused dequant GEMM, dX               */
   QLORA_K_GRAD = 6,         /* adapter gradients dA and dB (one     */
                             /* launch computes both)                */
-  QLORA_K_GRAD_REDUCE = 7,  /* unused: the split sums now happen    */
-                            /* inside the QLORA_K_GRAD launches     */
-  QLORA_K_SKINNY = 8        /* few-token forward                    */
+  QLORA_K_SKINNY = 7        /* few-token forward                    */
 } qlora_kernel_kind;
 
 qlora_status qlora_profile_enable(int on);

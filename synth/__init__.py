@@ -13,7 +13,7 @@ linear-layer workloads, W stored ``[N, K]`` = out x in):
 * ``llama7b``: W 4096x4096, 11008x4096, 4096x11008 ~N(0, 0.02), 4096 tokens,
                r=16, alpha=32, A ~N(0, 1/16), B ~N(0, 0.01).
 * ``skinny``:  W 4096x4096, 11008x4096, M in {1, 4, 16} tokens, r=16, fwd only.
-* ``llama65b``: W 8192x8192, 22016x8192 ~N(0, 0.015), 8192 tokens, r=64,
+* ``llama65b``: W 8192x8192, 22016x8192, 8192x22016 ~N(0, 0.015), 8192 tokens, r=64,
                alpha=16, A ~N(0, 1/64), B ~N(0, 0.01).
 * ``tensor1e9``: 1.0e9 bf16 ~N(0, 0.02), each element independently (p=1e-3)
                multiplied by 8 (heavy-tail outliers).
@@ -24,10 +24,12 @@ from .generators import (  # noqa: F401
     bf16_bits_from_f32,
     bf16_bits_to_f32,
     normal_bf16,
+    normal_bf16_rows,
     heavy_tail_chunk,
     CHUNK_ELEMS,
     n_chunks,
     linear_problem,
+    linear_problem_rows,
     LinearProblem,
     WORKLOADS,
 )

@@ -51,6 +51,38 @@ def normal_bf16(seed: int, tag: str, shape, std: float) -> np.ndarray:
     return out.reshape(shape)
 
 
+def normal_bf16_rows(seed: int, tag: str, shape, std: float, rows: int) -> np.ndarray:
+    """The first `rows` rows of ``normal_bf16(seed, tag, shape, std)`` (a 2-D shape),
+    bit for bit, drawing only the chunks that hold them."""
+    R, C = shape
+    rows = min(rows, R)
+    n = rows * C
+    out = np.empty(n, dtype=np.uint16)
+    tid = _tag_id(tag)
+    for c in range(0, (n + CHUNK_ELEMS - 1) // CHUNK_ELEMS):
+        lo = c * CHUNK_ELEMS
+        hi_full = min(R * C, lo + CHUNK_ELEMS)
+        g = np.random.default_rng([seed, tid, c])
+        z = g.standard_normal(hi_full - lo, dtype=np.float32)
+        hi = min(n, hi_full)
+        out[lo:hi] = bf16_bits_from_f32(z[: hi - lo] * np.float32(std))
+    return out.reshape(rows, C)
+
+
+def linear_problem_rows(M: int, N: int, K: int, r: int, alpha: float, w_std: float,
+                        tokens: int, wrows: int, seed: int = 0) -> LinearProblem:
+    """The leading part of ``linear_problem(M, N, K, r, alpha, w_std, seed)``: the
+    first `wrows` rows of W, the first `tokens` rows of X and dY, and A and B whole,
+    each bit-identical to the full problem's."""
+    tag = f"{M}x{N}x{K}r{r}"
+    W = normal_bf16_rows(seed, "W" + tag, (N, K), w_std, wrows)
+    X = normal_bf16_rows(seed, "X" + tag, (M, K), 1.0, tokens)
+    A = normal_bf16(seed, "A" + tag, (K, r), 1.0 / r)
+    B = normal_bf16(seed, "B" + tag, (r, N), 0.01)
+    dY = normal_bf16_rows(seed, "dY" + tag, (M, N), 1.0, tokens)
+    return LinearProblem(tag + f"[:{tokens}]", tokens, N, K, r, alpha, W, X, A, B, dY)
+
+
 def n_chunks(n: int) -> int:
     return (n + CHUNK_ELEMS - 1) // CHUNK_ELEMS
 
@@ -98,7 +130,7 @@ WORKLOADS: Dict[str, dict] = {
     "skinny": dict(w_std=0.02, r=16, alpha=32.0,
                    shapes=[(m, n, 4096) for n in (4096, 11008) for m in (1, 4, 16)]),
     "llama65b": dict(w_std=0.015, r=64, alpha=16.0,
-                     shapes=[(8192, 8192, 8192), (8192, 22016, 8192)]),
+                     shapes=[(8192, 8192, 8192), (8192, 22016, 8192), (8192, 8192, 22016)]),
 }
 
 

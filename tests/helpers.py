@@ -53,4 +53,32 @@ def bf16_ulp_check(got_bits: np.ndarray, ref: np.ndarray, contraction: int) -> f
     return float(np.max(np.abs(got - ref) / (ulp + rms_floor * rms)))
 
 
+# Element-wise bound of the fp32 rank-r outputs (XA, G, dA, dB), relative to the
+# matching product of magnitudes (for dA: s |X|^T |G|).  The operands of those
+# products are exact bf16 values or fp32 values carried as bf16 hi + lo pairs, which
+# represent them to 2^-17 relative; fp32 accumulation adds far less than that on
+# sums of random sign.  2^-15 leaves a factor 4.  A wrong row, column or split sum
+# shows up at order 1 / sqrt(contraction) of the magnitude, far above it.
+MAG_TOL = 2.0 ** -15
+
+
+def mag_check(got, ref, mag) -> float:
+    """Largest |got - ref| / (MAG_TOL * mag); <= 1 passes.  `mag` is the fp64
+    product of the operands' magnitudes for each output element."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    mag = np.asarray(mag, np.float64)
+    floor = 1e-30
+    return float(np.max(np.abs(got - ref) / (MAG_TOL * mag + floor)))
+
+
+def lora_magnitudes(X, A, B, dY, s, XA=None, G=None):
+    """Magnitude products for XA, G, dA and dB (fp64; inputs bf16 bits, or fp64 for
+    XA and G when given)."""
+    Xa, Aa, Ba, dYa = (np.abs(olin.as_f64(t)) for t in (X, A, B, dY))
+    XAm = np.abs(np.asarray(XA, np.float64)) if XA is not None else Xa @ Aa
+    Gm = np.abs(np.asarray(G, np.float64)) if G is not None else dYa @ Ba.T
+    return dict(XA=Xa @ Aa, G=dYa @ Ba.T, dA=abs(s) * (Xa.T @ Gm), dB=abs(s) * (XAm.T @ dYa))
+
+
 rel_fro = olin.rel_fro

@@ -6,7 +6,9 @@ outputs; bf16 rounding alone costs ~1.66e-3), and <= 1e-4 for the fp32
 outputs XA, dA and dB (fp32 accumulation over at most 8192 tokens; a bf16
 intermediate anywhere in those paths would show up as ~1e-3).  Y and dX are
 also checked element-wise: within one bf16 ulp of the exact value, with an
-absolute floor of 4 sqrt(K) 2^-23 rms for results that cancel to near zero."""
+absolute floor of 4 sqrt(K) 2^-23 rms for results that cancel to near zero.
+XA, dA and dB are checked element-wise too: within 2^-15 of the product of the
+operands' magnitudes (helpers.mag_check)."""
 import numpy as np
 import pytest
 
@@ -71,6 +73,11 @@ def _check(p, got, rows=None):
     assert errs["Y"] <= TOL_BF16, errs
     assert H.bf16_ulp_check(Yg, Y, p.K + 2 * p.r) <= 1.0, errs
     assert errs["XA"] <= TOL_FP32 and errs["dA"] <= TOL_FP32 and errs["dB"] <= TOL_FP32, errs
+    mag = H.lora_magnitudes(p.X, p.A, p.B, p.dY, p.s, XA=XA)
+    for k in ("XA", "dA", "dB"):
+        ref = XA if k == "XA" else g[k]
+        errs[k + "_mag"] = H.mag_check(got[k], ref, mag[k])
+        assert errs[k + "_mag"] <= 1.0, (k, errs)
     if dXg is not None:
         errs["dX"] = olin.rel_fro(H.onf4.bf16_to_f32(dXg), g["dX"])
         assert errs["dX"] <= TOL_BF16, errs
@@ -128,6 +135,30 @@ def test_linear_llama65b_shapes_sampled_rows(q, N, K):
     _check(p, got, rows=rows)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(384, 256, 384, 16), (256, 640, 256, 64)])
+def test_projection_G_direct(q, M, N, K, r):
+    """G = dY B^T checked on its own: with X = the first K rows of the identity
+    (M = K tokens, the rest zero), dA = s X^T G is s G[k, :] for k < K, carried
+    through the gradient kernel as bf16 hi + lo, i.e. to 2^-17 relative.  So
+    every element of s G is compared with the oracle's, within 2^-15 of its
+    magnitude product s |dY| |B|^T."""
+    import torch
+    p = linear_problem(M, N, K, r, 2.0 * r, 0.02, seed=21)
+    Xi = np.zeros((M, K), np.uint16)
+    Xi[np.arange(min(M, K)), np.arange(min(M, K))] = 0x3F80          # bf16 1.0
+    X = H.bits_to_dev(Xi)
+    Wq = q.nf4_quantize(H.bits_to_dev(p.W))
+    A, B, dY = H.bits_to_dev(p.A), H.bits_to_dev(p.B), H.bits_to_dev(p.dY)
+    _, dA, _ = q.linear_bwd(dY, X, None, Wq, A, B, p.s, need_dx=False)
+    torch.cuda.synchronize()
+    assert q.device_status() == (0, 0)
+    G = olin.as_f64(p.dY) @ olin.as_f64(p.B).T
+    n = min(M, K)
+    got = dA.cpu().numpy().astype(np.float64)[:n]
+    mag = abs(p.s) * (np.abs(olin.as_f64(p.dY)) @ np.abs(olin.as_f64(p.B)).T)[:n]
+    assert H.mag_check(got, p.s * G[:n], mag) <= 1.0
+
+
 @pytest.mark.parametrize("N,K", [(256, 384), (384, 256), (128, 1024)])
 def test_gemm_dequant_bit_exact_one_hot(q, N, K):
     """With X = I (K one-hot tokens) and A = 0 every output of the forward is a
@@ -153,9 +184,8 @@ def test_gemm_dequant_bit_exact_one_hot(q, N, K):
 
 
 def test_fwd_bwd_capture_in_cuda_graph(q):
-    """The forward and backward (which fork the block-constant expansion onto the
-    library's side stream and join it back) capture into one CUDA graph; replays
-    give bit-identical results to eager calls."""
+    """The forward and backward capture into one CUDA graph; replays give
+    bit-identical results to eager calls."""
     import torch
     p = linear_problem(64, 384, 512, 16, 32.0, 0.02, seed=3)
     X, A, B, dY = (H.bits_to_dev(v) for v in (p.X, p.A, p.B, p.dY))
@@ -186,6 +216,53 @@ def test_fwd_bwd_capture_in_cuda_graph(q):
     for got, want in zip((Y, XA, dX, dA, dB), ref):
         assert torch.equal(got.view(torch.int16) if got.dtype == torch.bfloat16 else got.view(torch.int32),
                            want.view(torch.int16) if want.dtype == torch.bfloat16 else want.view(torch.int32))
+
+
+def test_graph_replay_with_new_inputs_at_a_split_shape(q):
+    """4096 tokens on a 4096 x 4096 weight make 512 GEMM tiles on 148 SMs: the 68
+    tiles of the last round are split in contraction halves in both the forward
+    and the dX GEMM.  A forward + backward captured once and replayed with new X
+    and dY in the same buffers must give, bit for bit, what eager calls give on
+    those inputs (the split tiles' arrival counters must start from zero on every
+    replay)."""
+    import torch
+    M, N, K, r = 4096, 4096, 4096, 16
+    ps = [linear_problem(M, N, K, r, 32.0, 0.02, seed=sd) for sd in (31, 32, 33)]
+    Wq = q.nf4_quantize(H.bits_to_dev(ps[0].W))
+    A, B = H.bits_to_dev(ps[0].A), H.bits_to_dev(ps[0].B)
+    X = H.bits_to_dev(ps[0].X)
+    dY = H.bits_to_dev(ps[0].dY)
+    ws = q.make_workspace(M, N, K, r, X.device)
+    outs = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(M, r, dtype=torch.float32, device="cuda"),
+            torch.empty(M, K, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(K, r, dtype=torch.float32, device="cuda"),
+            torch.empty(r, N, dtype=torch.float32, device="cuda")]
+    s = ps[0].s
+
+    def step(Xt, dYt, Y, XA, dX, dA, dB):
+        q.linear_fwd(Xt, Wq, A, B, s, workspace=ws, Y=Y, XA=XA)
+        q.linear_bwd(dYt, Xt, XA, Wq, A, B, s, workspace=ws, dX=dX, dA=dA, dB=dB)
+
+    step(X, dY, *outs)                                  # eager warm-up on the first inputs
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(X, dY, *outs)
+    for p in ps[1:]:
+        X.copy_(H.bits_to_dev(p.X))
+        dY.copy_(H.bits_to_dev(p.dY))
+        g.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in outs]
+        ref = [torch.empty_like(t) for t in outs]
+        step(X, dY, *ref)
+        torch.cuda.synchronize()
+        assert q.device_status() == (0, 0)
+        for a, b in zip(got, ref):
+            assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                               b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
+    del g
 
 
 @pytest.mark.gpu

@@ -3,7 +3,8 @@ the NF4 weight decoded in registers) against the fp64 oracle.
 
 Bars as in test_gpu_linear: relative Frobenius <= 2e-3 for Y (bf16 output) and
 <= 1e-4 for the fp32 XA; Y also element-wise within one bf16 ulp (plus the
-accumulation floor for near-zero results).  The dequantization inside the
+accumulation floor for near-zero results), XA element-wise within 2^-15 of
+|X| |A|.  The dequantization inside the
 kernel is checked bit for bit with one-hot tokens."""
 import numpy as np
 import pytest
@@ -40,6 +41,8 @@ def _check(p, Yb, XA):
     ex = olin.rel_fro(XA, XAr)
     assert ey <= 2e-3 and ex <= 1e-4, (ey, ex)
     assert H.bf16_ulp_check(Yb, Y, p.K + p.r) <= 1.0
+    mag = np.abs(olin.as_f64(p.X)) @ np.abs(olin.as_f64(p.A))
+    assert H.mag_check(XA, XAr, mag) <= 1.0
     return ey, ex
 
 

@@ -43,3 +43,17 @@ def test_distributions():
     # |z| > 0.75, i.e. 45% of the time, so ~4.5e-4 of the values (+-1e-5 at this size)
     frac = np.mean(np.abs(h) > 6 * 0.02)
     assert 3.5e-4 < frac < 5.5e-4
+
+
+def test_row_prefix_generators_match_the_full_tensors():
+    """normal_bf16_rows / linear_problem_rows give the leading rows of the full
+    tensors bit for bit, also when the rows span more than one seeded chunk."""
+    from synth import CHUNK_ELEMS, linear_problem, linear_problem_rows, normal_bf16, normal_bf16_rows
+    full = normal_bf16(3, "prefix", (3000, 8192), 0.5)
+    rows = CHUNK_ELEMS // 8192 + 52                  # crosses the first chunk boundary
+    assert np.array_equal(normal_bf16_rows(3, "prefix", (3000, 8192), 0.5, rows), full[:rows])
+    assert np.array_equal(normal_bf16_rows(3, "prefix", (3000, 8192), 0.5, 5000), full)
+    p = linear_problem(40, 96, 128, 8, 16.0, 0.02, seed=2)
+    s = linear_problem_rows(40, 96, 128, 8, 16.0, 0.02, 7, 33, seed=2)
+    assert np.array_equal(s.W, p.W[:33]) and np.array_equal(s.X, p.X[:7])
+    assert np.array_equal(s.dY, p.dY[:7]) and np.array_equal(s.A, p.A) and np.array_equal(s.B, p.B)
