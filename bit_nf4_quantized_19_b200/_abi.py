@@ -56,13 +56,20 @@ SIGNATURES = {
     "qlora_status_string": (ctypes.c_char_p, [_int]),
     "qlora_nf4_levels": (None, [ctypes.POINTER(ctypes.c_float)]),
     "qlora_nf4_bytes": (_sz, [_i64, _i64, _szp, _szp, _szp]),
+    "qlora_nf4_single_bytes": (_sz, [_i64, _i64, _szp, _szp]),
     "qlora_nf4_quantize": (_int, [_vp, _i64, _i64, _nf4p, _vp]),
     "qlora_nf4_dequant": (_int, [_nf4p, _vp, _vp]),
     "qlora_linear_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_fwd_ex": (_int, [_vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _f32, _vp, _vp, _vp, _sz,
+                                   _vp]),
+    "qlora_linear_dropout_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "qlora_linear_fwd_noalloc": (_int, [_vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _vp, _vp,
                                 _vp, _sz, _vp]),
+    "qlora_linear_bwd_ex": (_int, [_vp, _vp, _vp, _i64, _nf4p, _vp, _vp, _int, _f32, _vp, _f32, _int, _vp,
+                                   _vp, _vp, _vp, _sz, _vp]),
+    "qlora_nf4_merge": (_int, [_nf4p, _vp, _i64, _i64, _vp, _vp, _int, _f32, _vp, _vp]),
     "qlora_get_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "qlora_selftest_wait_timeout": (_int, [_u32, _vp]),
     "qlora_set_wait_limit_us": (_u32, [_u32]),
@@ -71,7 +78,7 @@ SIGNATURES = {
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "prep", "project", "gemm_fwd", "gemm_dx",
-                "grad", "skinny"]
+                "grad", "skinny", "merge"]
 PROFILE_CAP = 4096
 
 _LIB = None

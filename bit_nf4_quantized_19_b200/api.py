@@ -32,20 +32,26 @@ def _bf16_2d(t: torch.Tensor, name: str) -> torch.Tensor:
 @dataclasses.dataclass
 class NF4Weight:
     """A quantized frozen weight [rows, cols]: packed codes, 8-bit block
-    constants, fp32 group constants (device tensors owned by this object)."""
+    constants, fp32 group constants (device tensors owned by this object).  With
+    q8 = None the constants are single-level: `step` holds one fp32 absmax per
+    64-value block."""
     codes: torch.Tensor
-    q8: torch.Tensor
+    q8: Optional[torch.Tensor]
     step: torch.Tensor
     rows: int
     cols: int
 
     def c_struct(self) -> _abi.NF4Struct:
-        return _abi.NF4Struct(self.codes.data_ptr(), self.q8.data_ptr(), self.step.data_ptr(),
-                              self.rows, self.cols)
+        return _abi.NF4Struct(self.codes.data_ptr(), self.q8.data_ptr() if self.q8 is not None else None,
+                              self.step.data_ptr(), self.rows, self.cols)
+
+    @property
+    def single_level(self) -> bool:
+        return self.q8 is None
 
     @property
     def nbytes(self) -> int:
-        return self.codes.numel() + self.q8.numel() + 4 * self.step.numel()
+        return self.codes.numel() + (self.q8.numel() if self.q8 is not None else 0) + 4 * self.step.numel()
 
 
 def nf4_levels() -> list:
@@ -67,11 +73,23 @@ def nf4_empty(rows: int, cols: int, device) -> NF4Weight:
                      torch.empty(sb // 4, dtype=torch.float32, device=device), rows, cols)
 
 
-def nf4_quantize(W: torch.Tensor, out: Optional[NF4Weight] = None) -> NF4Weight:
-    """Blockwise NF4 + double quantization of a bf16 [rows, cols] CUDA tensor."""
+def nf4_empty_single(rows: int, cols: int, device) -> NF4Weight:
+    """Storage for single-level constants (one fp32 absmax per 64-value block)."""
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _abi.lib().qlora_nf4_single_bytes(rows, cols, ctypes.byref(c), ctypes.byref(s))
+    return NF4Weight(torch.empty(c.value, dtype=torch.uint8, device=device), None,
+                     torch.empty(s.value // 4, dtype=torch.float32, device=device), rows, cols)
+
+
+def nf4_quantize(W: torch.Tensor, out: Optional[NF4Weight] = None, single_level: bool = False) -> NF4Weight:
+    """Blockwise NF4 quantization of a bf16 [rows, cols] CUDA tensor, with
+    double-quantized constants (default) or single-level fp32 ones."""
     W = _bf16_2d(W, "W")
     rows, cols = W.shape
-    q = out if out is not None else nf4_empty(rows, cols, W.device)
+    if out is not None:
+        q = out
+    else:
+        q = nf4_empty_single(rows, cols, W.device) if single_level else nf4_empty(rows, cols, W.device)
     st = q.c_struct()
     _abi.check(_abi.lib().qlora_nf4_quantize(_ptr(W), rows, cols, ctypes.byref(st),
                                              _stream(W.device)), "qlora_nf4_quantize")
@@ -87,12 +105,25 @@ def nf4_dequant(Wq: NF4Weight, out: Optional[torch.Tensor] = None) -> torch.Tens
     return out
 
 
-def workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+def workspace_bytes(M: int, N: int, K: int, r: int, dropout: bool = False) -> int:
+    if dropout:
+        return int(_abi.lib().qlora_linear_dropout_workspace_bytes(M, N, K, r))
     return int(_abi.lib().qlora_linear_workspace_bytes(M, N, K, r))
 
 
-def make_workspace(M: int, N: int, K: int, r: int, device) -> torch.Tensor:
-    return torch.empty(workspace_bytes(M, N, K, r), dtype=torch.uint8, device=device)
+def make_workspace(M: int, N: int, K: int, r: int, device, dropout: bool = False) -> torch.Tensor:
+    return torch.empty(workspace_bytes(M, N, K, r, dropout), dtype=torch.uint8, device=device)
+
+
+def pack_keep_mask(keep: torch.Tensor) -> torch.Tensor:
+    """A boolean [M, K] keep mask as the library's bit-packed form: element m K + k in
+    bit (m K + k) mod 8 of byte (m K + k) / 8 (uint8 [M K / 8], on keep's device).
+    Marshalling only (torch bit operations)."""
+    if keep.dim() != 2 or keep.shape[1] % 8:
+        raise ValueError("keep must be [M, K] with K a multiple of 8")
+    bits = keep.reshape(-1, 8).to(torch.uint8)
+    w = torch.tensor([1, 2, 4, 8, 16, 32, 64, 128], dtype=torch.uint8, device=keep.device)
+    return (bits * w).sum(dim=1, dtype=torch.uint8).contiguous()
 
 
 def _check_shapes(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor,
@@ -108,8 +139,11 @@ def _check_shapes(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tens
 
 def linear_fwd(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, s: float,
                workspace: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
-               XA: Optional[torch.Tensor] = None, want_xa: bool = True):
-    """Y = X deq(W)^T + s (X A) B  (bf16 [M, N]);  returns (Y, XA fp32 [M, r] or None)."""
+               XA: Optional[torch.Tensor] = None, want_xa: bool = True,
+               keep_bits: Optional[torch.Tensor] = None, dropout_p: float = 0.0):
+    """Y = X deq(W)^T + s (X A) B  (bf16 [M, N]);  returns (Y, XA fp32 [M, r] or None).
+    With keep_bits (pack_keep_mask of the [M, K] keep mask) the adapter input is
+    X (.) keep / (1 - dropout_p)."""
     X = _bf16_2d(X, "X")
     A = _bf16_2d(A, "A")
     B = _bf16_2d(B, "B")
@@ -122,19 +156,27 @@ def linear_fwd(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor,
     if XA is None and want_xa:
         XA = torch.empty(M, r, dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = make_workspace(M, Wq.rows, Wq.cols, r, dev)
+        workspace = make_workspace(M, Wq.rows, Wq.cols, r, dev, dropout=keep_bits is not None)
     st = Wq.c_struct()
-    _abi.check(_abi.lib().qlora_linear_fwd(
-        _ptr(X), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(XA),
-        _ptr(workspace), workspace.numel(), _stream(dev)), "qlora_linear_fwd")
+    if keep_bits is None:
+        _abi.check(_abi.lib().qlora_linear_fwd(
+            _ptr(X), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(XA),
+            _ptr(workspace), workspace.numel(), _stream(dev)), "qlora_linear_fwd")
+    else:
+        _abi.check(_abi.lib().qlora_linear_fwd_ex(
+            _ptr(X), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s), _ptr(keep_bits), float(dropout_p),
+            _ptr(Y), _ptr(XA), _ptr(workspace), workspace.numel(), _stream(dev)), "qlora_linear_fwd_ex")
     return Y, XA
 
 
 def linear_bwd(dY: torch.Tensor, X: torch.Tensor, XA: Optional[torch.Tensor], Wq: NF4Weight,
                A: torch.Tensor, B: torch.Tensor, s: float, need_dx: bool = True,
                workspace: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,
-               dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None):
-    """Returns (dX bf16 [M, K] or None, dA fp32 [K, r], dB fp32 [r, N])."""
+               dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+               keep_bits: Optional[torch.Tensor] = None, dropout_p: float = 0.0,
+               accumulate: bool = False):
+    """Returns (dX bf16 [M, K] or None, dA fp32 [K, r], dB fp32 [r, N]).  keep_bits /
+    dropout_p as in linear_fwd; accumulate adds into the given dA and dB."""
     dY = _bf16_2d(dY, "dY")
     X = _bf16_2d(X, "X")
     A = _bf16_2d(A, "A")
@@ -149,14 +191,50 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, XA: Optional[torch.Tensor], Wq
         dA = torch.empty(Wq.cols, r, dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty(r, Wq.rows, dtype=torch.float32, device=dev)
+    if accumulate and (dA is None or dB is None):
+        raise ValueError("accumulate needs the dA and dB to add into")
     if workspace is None:
-        workspace = make_workspace(M, Wq.rows, Wq.cols, r, dev)
+        workspace = make_workspace(M, Wq.rows, Wq.cols, r, dev, dropout=keep_bits is not None)
     st = Wq.c_struct()
-    _abi.check(_abi.lib().qlora_linear_bwd(
-        _ptr(dY), _ptr(X), _ptr(XA), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s),
-        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream(dev)),
-        "qlora_linear_bwd")
+    if keep_bits is None and not accumulate:
+        _abi.check(_abi.lib().qlora_linear_bwd(
+            _ptr(dY), _ptr(X), _ptr(XA), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s),
+            _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream(dev)),
+            "qlora_linear_bwd")
+    else:
+        _abi.check(_abi.lib().qlora_linear_bwd_ex(
+            _ptr(dY), _ptr(X), _ptr(XA), M, ctypes.byref(st), _ptr(A), _ptr(B), r, float(s),
+            _ptr(keep_bits), float(dropout_p), 1 if accumulate else 0,
+            _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream(dev)),
+            "qlora_linear_bwd_ex")
     return dX, dA, dB
+
+
+def nf4_merge(A: torch.Tensor, B: torch.Tensor, s: float, Wq: Optional[NF4Weight] = None,
+              W16: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The adapter folded into a 16-bit weight: bf16(base + s (A B)^T) [N, K], base the
+    bf16 original W16 or the dequantized Wq (pass exactly one)."""
+    A = _bf16_2d(A, "A")
+    B = _bf16_2d(B, "B")
+    if (Wq is None) == (W16 is None):
+        raise ValueError("pass exactly one of Wq and W16")
+    if W16 is not None:
+        W16 = _bf16_2d(W16, "W16")
+        N, K = W16.shape
+        dev = W16.device
+    else:
+        N, K = Wq.rows, Wq.cols
+        dev = Wq.codes.device
+    r = A.shape[1]
+    if A.shape[0] != K or tuple(B.shape) != (r, N):
+        raise ValueError(f"shape mismatch: W [{N}, {K}], A {tuple(A.shape)}, B {tuple(B.shape)}")
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    st = Wq.c_struct() if Wq is not None else None
+    _abi.check(_abi.lib().qlora_nf4_merge(ctypes.byref(st) if st is not None else None, _ptr(W16), N, K,
+                                          _ptr(A), _ptr(B), r, s, _ptr(out), _stream(dev)),
+               "qlora_nf4_merge")
+    return out
 
 
 def device_status(sync_stream: bool = True) -> Tuple[int, int]:

@@ -16,7 +16,8 @@ LIB_NAME = "libqlora_nf4.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
 SOURCES = ["qlora_nf4.cu", "nf4_table.cpp"]
-HEADERS = ["common.cuh", "gemm_kernel.cuh", "lora_mma.cuh", "quant_kernels.cuh", "skinny_kernel.cuh",
+HEADERS = ["common.cuh", "gemm_kernel.cuh", "lora_mma.cuh", "merge_kernel.cuh", "quant_kernels.cuh",
+           "skinny_kernel.cuh",
            "nf4_table.hpp"]
 
 NVCC_FLAGS = [

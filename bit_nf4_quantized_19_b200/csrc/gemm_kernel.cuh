@@ -67,6 +67,10 @@ constexpr int kBStageBytes = kBN * 128;   // 32 KB
 constexpr int kAStageBytes = kWT * 128;   // 16 KB
 constexpr int kWStageBytes = 4096;        // packed codes of one stage
 constexpr int kSStageBytes = 512;         // 128 fp32 block constants of one stage
+#ifndef QLORA_GEMM_SCALE_PRE
+#define QLORA_GEMM_SCALE_PRE 6
+#endif
+constexpr int kScalePre = QLORA_GEMM_SCALE_PRE;   // stages of block constants requested ahead
 constexpr uint32_t kSplitArrive = 1u;     // split-tile counter: one per arriving half
 constexpr uint32_t kSplitReady = 16u;     // added once the first half's partial is stored
 constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
@@ -89,8 +93,8 @@ struct GemmParams {
   int r;
   int lora_ld;       // row pitch of the LoRA weight operand source: N (B [r,N]) or r (A [K,r])
   int KB;            // 64-value blocks per weight row: K / 64
-  const uint8_t *q8;       // 8-bit block constants of W, [N * KB]
-  const float *step;       // fp32 group constants, one per 256 blocks
+  const uint8_t *q8;       // 8-bit block constants of W, [N * KB]; null: single-level
+  const float *step;       // fp32 group constants, one per 256 blocks (single-level: one per block)
   const uint16_t *lora_w;  // fwd: B [r, N];  dX: A [K, r]
   uint16_t *out;     // Y [M, N] or dX [M, K]
   uint64_t limit_ns;
@@ -99,6 +103,11 @@ struct GemmParams {
   int kb_mid;        // first main stage of the second half
   float *scratch;    // [split_count][128][256] fp32 partial tile of the half that finishes first
   unsigned int *flags;   // [split_count] arrival counters, zero at launch
+  // dX under adapter-input dropout (null otherwise): the keep mask of X [M, K], bit-packed
+  // (element m K + k in bit (m K + k) mod 32 of word (m K + k) / 32).  The adapter term
+  // then gets its own accumulator and is added as keep * keep_scale * term per element.
+  const uint32_t *keep32;
+  float keep_scale;      // 1 / (1 - p)
   float levels[16];
 };
 
@@ -152,8 +161,14 @@ QDEV void load_stage_scales(const GemmParams &p, int w0, int kb, int lane, uint3
     int64_t b;
     if (MODE == kModeFwd) b = static_cast<int64_t>(w0 + idx) * p.KB + kb;
     else b = static_cast<int64_t>(kb * kBK + (idx & 63)) * p.KB + (w0 >> 6) + (idx >> 6);
-    q[i] = __ldg(p.q8 + b);
-    st[i] = __ldg(p.step + (b >> 8));
+    if (p.q8) {
+      q[i] = __ldg(p.q8 + b);
+      st[i] = __ldg(p.step + (b >> 8));
+    } else {
+      // single-level constants: the block's own fp32 absmax, and RN32(1 * a_b) = a_b
+      q[i] = 1u;
+      st[i] = __ldg(p.step + b);
+    }
   }
 }
 QDEV void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -251,30 +266,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ weight producer
+    // The raw constants of a stage are requested kScalePre stages before it is
+    // produced (a lookahead iterator runs that far ahead of the ring), so their L2
+    // latency stays off the producer's path.
     int ws = 0;
     uint32_t wph = 0;
     uint32_t armedW = 0, lastW = 0;
-    GemmItem w;
-    int it = 0;
+    GemmItem w, wa;
+    int it = 0, ita = 0;
     bool have = gemm_item(p, num_tiles, 0, w);
     int kb = have ? w.kb0 : 0;
-    uint32_t q_cur[4] = {0u, 0u, 0u, 0u};
-    float s_cur[4] = {0.f, 0.f, 0.f, 0.f};
-    if (have) load_stage_scales<MODE>(p, (w.tile % p.num_w_tiles) * kWT, kb, lane, q_cur, s_cur);
+    bool have_a = have;
+    wa = w;
+    int kba = kb;
+    auto advance_a = [&]() {
+      if (!have_a) return;
+      if (++kba >= wa.kb1) {
+        ++ita;
+        have_a = gemm_item(p, num_tiles, ita, wa);
+        kba = have_a ? wa.kb0 : 0;
+      }
+    };
+    uint32_t qv[kScalePre][4];
+    float sv[kScalePre][4];
+#pragma unroll
+    for (int d = 0; d < kScalePre; ++d) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { qv[d][i] = 0u; sv[d][i] = 0.f; }
+      if (have_a) load_stage_scales<MODE>(p, (wa.tile % p.num_w_tiles) * kWT, kba, lane, qv[d], sv[d]);
+      advance_a();
+    }
     while (have) {
       const int w0 = (w.tile % p.num_w_tiles) * kWT;
-      // the next stage's raw constants are requested now and used one iteration later
-      GemmItem wn = w;
-      int itn = it, kbn = kb + 1;
-      bool have_n = true;
-      if (kbn >= w.kb1) {
-        itn = it + 1;
-        have_n = gemm_item(p, num_tiles, itn, wn);
-        kbn = have_n ? wn.kb0 : 0;
-      }
-      uint32_t q_nxt[4] = {0u, 0u, 0u, 0u};
-      float s_nxt[4] = {0.f, 0.f, 0.f, 0.f};
-      if (have_n) load_stage_scales<MODE>(p, (wn.tile % p.num_w_tiles) * kWT, kbn, lane, q_nxt, s_nxt);
       // warp-uniform: every lane arrives on full_W below
       if (!__all_sync(0xffffffffu, wait_bar(&empty_W[ws], wph ^ 1u, wt))) break;
       if (lane == 0) {
@@ -291,15 +314,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        sS[ws * 128 + lane + 32 * i] = __fmul_rn(static_cast<float>(q_cur[i]), s_cur[i]);
+        sS[ws * 128 + lane + 32 * i] = __fmul_rn(static_cast<float>(qv[0][i]), sv[0][i]);
       mbar_arrive(&full_W[ws]);
       if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
-      w = wn;
-      it = itn;
-      kb = kbn;
-      have = have_n;
+      // shift the prefetch ring and request the stage kScalePre ahead
 #pragma unroll
-      for (int i = 0; i < 4; ++i) { q_cur[i] = q_nxt[i]; s_cur[i] = s_nxt[i]; }
+      for (int d = 0; d + 1 < kScalePre; ++d) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { qv[d][i] = qv[d + 1][i]; sv[d][i] = sv[d + 1][i]; }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { qv[kScalePre - 1][i] = 0u; sv[kScalePre - 1][i] = 0.f; }
+      if (have_a)
+        load_stage_scales<MODE>(p, (wa.tile % p.num_w_tiles) * kWT, kba, lane, qv[kScalePre - 1],
+                                sv[kScalePre - 1]);
+      advance_a();
+      // next stage
+      if (++kb >= w.kb1) {
+        ++it;
+        have = gemm_item(p, num_tiles, it, w);
+        kb = have ? w.kb0 : 0;
+      }
     }
     if (lane == 0) {
       volatile int no_abort = 0;
@@ -324,6 +359,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t bd0 = sw128_desc(b0, 16, 1024);
       const int kb_lora = p.kb_lora;
       const int lora_steps_total = (2 * p.r) / 16;
+      // under dropout (dX only) one tile at a time: main product in columns [0, 256),
+      // adapter term in [256, 512)
+      const bool two_acc = (MODE == kModeDx) && (p.keep32 != nullptr);
+      const int nacc = two_acc ? 1 : 2;
       int st = 0, acc = 0;
       uint32_t ph = 0, accph = 0;
       bool ok = true;
@@ -332,6 +371,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!wait_bar(&tmem_empty[acc], accph ^ 1u, wt)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        const uint32_t d_lora = two_acc ? tmem_base + static_cast<uint32_t>(kBN) : d_tmem;
         for (int kb = 0; kb < w.kb1 - w.kb0; ++kb) {
           if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
@@ -350,13 +390,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStageBytes >> 4));
           const int nk = min(4, lora_steps_total - ls * 4);
           for (int k = 0; k < nk; ++k)
-            mma_bf16_ss(d_tmem, ad + k * a_step_lora, bd + k * 2, idesc_lora, 1u);
+            mma_bf16_ss(d_lora, ad + k * a_step_lora, bd + k * 2, idesc_lora,
+                        (two_acc && (ls | k) == 0) ? 0u : 1u);
           mma_commit(&empty_A[st]);
           if (++st == kStagesA) { st = 0; ph ^= 1u; }
         }
         if (!ok) break;
         mma_commit(&tmem_full[acc]);
-        if (++acc == 2) { acc = 0; accph ^= 1u; }
+        if (++acc == nacc) { acc = 0; accph ^= 1u; }
       }
       // All issued MMAs complete before TMEM is released (bounded).
       mma_commit(drain);
@@ -368,6 +409,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;      // weight-side row within the tile
+    const bool two_acc = (MODE == kModeDx) && (p.keep32 != nullptr);
+    const int nacc = two_acc ? 1 : 2;
+    const int64_t keep_words = static_cast<int64_t>(p.n_out) >> 5;   // mask words per token
     int acc = 0;
     uint32_t accph = 0;
     GemmItem w;
@@ -411,6 +455,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                static_cast<uint32_t>(acc * kBN + cc * 32),
                            v);
         tmem_wait_ld();
+        if (two_acc && w.lora) {
+          // this tile's contribution: main + keep * (1/(1-p)) * adapter term, per element;
+          // the warp's 32 rows are 32 consecutive input features, one mask word per token
+          const int mb = m0 + cc * 32;
+          const int64_t kw = (w0 + q * 32) >> 5;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t lv[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(kBN + cc * 32 + h * 16),
+                               lv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int m = mb + h * 16 + j;
+              const uint32_t word = (m < p.M) ? __ldg(p.keep32 + static_cast<int64_t>(m) * keep_words + kw) : 0u;
+              if ((word >> lane) & 1u)
+                v[h * 16 + j] = __float_as_uint(__fadd_rn(__uint_as_float(v[h * 16 + j]),
+                                                          __fmul_rn(p.keep_scale, __uint_as_float(lv[j]))));
+            }
+          }
+        }
         if (role == 1) {
           float4 *d4 = reinterpret_cast<float4 *>(prow + cc * 32);
 #pragma unroll
@@ -449,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tmem_empty[acc]);
-      if (++acc == 2) { acc = 0; accph ^= 1u; }
+      if (++acc == nacc) { acc = 0; accph ^= 1u; }
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequant producers

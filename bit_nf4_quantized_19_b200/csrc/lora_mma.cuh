@@ -58,6 +58,10 @@ struct LoraMmaParams {
   // split-tile arrival counters); CTA (0, 0) clears them.  May be null.
   unsigned int *zero;
   int zero_n;
+  // Factor applied to the fp32 result before it is stored (1/(1-p) for products over
+  // the dropped-out adapter input), for the first and the second product.
+  float out_scale, out_scale1;
+  int accumulate;        // gradients: add into out instead of overwriting it
 };
 
 constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of a tile
@@ -104,6 +108,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   const int rows = second ? p.rows1 : p.rows;
   float *const out = second ? p.out1 : p.out;
   const int layout = second ? p.layout1 : p.layout;
+  const float out_scale = second ? p.out_scale1 : p.out_scale;
   const CUtensorMap *const map_act = second ? &tm_act1 : &tm_act;
   const CUtensorMap *const map_q = second ? &tm_q1 : &tm_q;
   const int split = blockIdx.y;
@@ -237,12 +242,14 @@ __global__ void __launch_bounds__(kLmThreads, 1)
 #pragma unroll
         for (int qq = 0; qq < kLmClusterMax; ++qq)
           if (qq < p.splits) v += pa[qq] + pb[qq];
-        if (layout == 0) out[static_cast<int64_t>(row) * p.r + j] = v;
-        else out[static_cast<int64_t>(j) * rows + row] = v;
+        v = __fmul_rn(v, out_scale);
+        float *o = (layout == 0) ? out + static_cast<int64_t>(row) * p.r + j : out + static_cast<int64_t>(j) * rows + row;
+        *o = p.accumulate ? __fadd_rn(*o, v) : v;
       } else {
 #pragma unroll
         for (int qq = 0; qq < kLmClusterMax; ++qq)
           if (qq < p.splits) v += pa[qq];
+        v = __fmul_rn(v, out_scale);
         if (out) out[static_cast<int64_t>(row) * p.r + j] = v;
         uint16_t h, l;
         split_hilo(p.s * v, h, l);
@@ -269,6 +276,26 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__r
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t j = i / K, k = i - j * K;
     AT[i] = A[k * r + j];
+  }
+}
+
+// Xd = X (.) keep: the adapter input with its dropped elements set to zero (exact in
+// bf16).  keep is a bit-packed mask of the n = M K elements, element e in bit e mod 8
+// of byte e / 8; n is a multiple of 8.  Eight elements (16 bytes) per thread and step.
+__global__ void __launch_bounds__(256) mask_input_kernel(const uint16_t *__restrict__ X,
+                                                         const uint8_t *__restrict__ keep, int64_t n8,
+                                                         uint16_t *__restrict__ Xd) {
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n8;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 x = ld_global_nc_v4(X + 8 * u);
+    const uint32_t b = keep[u];
+    // bit 2i keeps the low half of word i, bit 2i+1 the high half
+    auto m = [b](uint32_t w, int i) {
+      const uint32_t lo = ((b >> (2 * i)) & 1u) ? 0x0000FFFFu : 0u;
+      const uint32_t hi = ((b >> (2 * i + 1)) & 1u) ? 0xFFFF0000u : 0u;
+      return w & (lo | hi);
+    };
+    *reinterpret_cast<uint4 *>(Xd + 8 * u) = make_uint4(m(x.x, 0), m(x.y, 1), m(x.z, 2), m(x.w, 3));
   }
 }
 

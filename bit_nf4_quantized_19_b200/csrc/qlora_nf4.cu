@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "gemm_kernel.cuh"
 #include "lora_mma.cuh"
+#include "merge_kernel.cuh"
 #include "nf4_table.hpp"
 #include "quant_kernels.cuh"
 #include "skinny_kernel.cuh"
@@ -82,7 +83,9 @@ qlora_status device_info(DeviceInfo **out) {
             cudaSuccess ||
         set_skinny_attrs<1>() != cudaSuccess || set_skinny_attrs<2>() != cudaSuccess ||
         set_skinny_attrs<4>() != cudaSuccess || set_skinny_attrs<8>() != cudaSuccess ||
-        set_skinny_attrs<16>() != cudaSuccess)
+        set_skinny_attrs<16>() != cudaSuccess ||
+        cudaFuncSetAttribute(nf4_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             merge_smem_bytes(2)) != cudaSuccess)
       return QLORA_ERR_CUDA;
     d.gemm_attr_set = true;
   }
@@ -332,9 +335,10 @@ bool take_split(Workspace &ws, const GemmSplit &g, SplitScratch &out) {
 }
 
 qlora_status check_nf4(const qlora_nf4_t *Wq) {
-  if (!Wq || !Wq->codes || !Wq->q8 || !Wq->step) return QLORA_ERR_INVALID_ARG;
+  if (!Wq || !Wq->codes || !Wq->step) return QLORA_ERR_INVALID_ARG;   // q8 null: single-level constants
   if (Wq->rows <= 0 || Wq->cols <= 0) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(Wq->codes) || !aligned16(Wq->q8) || !aligned16(Wq->step)) return QLORA_ERR_MISALIGNED;
+  if (!aligned16(Wq->codes) || (Wq->q8 && !aligned16(Wq->q8)) || !aligned16(Wq->step))
+    return QLORA_ERR_MISALIGNED;
   return QLORA_OK;
 }
 
@@ -422,10 +426,14 @@ qlora_status launch_lora_mma(const LmOperands &o, int64_t contraction, int nn, L
 }
 
 // XA = X A (or G = dY B^T): fp32 [M, r] plus hi/lo of s*result in [M, 2r] and/or [2r, pad8(M)].
+// The fp32 result is multiplied by out_scale before it is stored and split (1/(1-p) for
+// the product over a dropped-out adapter input).
 qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const uint16_t *qT,
                                int r, float s, float *out, uint16_t *hl, uint16_t *hlT, int sms,
-                               cudaStream_t st, const SplitScratch *clear = nullptr) {
+                               cudaStream_t st, const SplitScratch *clear = nullptr,
+                               float out_scale = 1.0f) {
   LoraMmaParams p{};
+  p.out_scale = p.out_scale1 = out_scale;
   if (clear && clear->g.count) {
     p.zero = clear->flags;
     p.zero_n = clear->g.count;
@@ -450,13 +458,18 @@ qlora_status launch_hilo_t(const float *v, int64_t M, int r, float s, uint16_t *
 }
 
 // Both adapter gradients in one launch, each act^T * (hi + lo) over the M tokens:
-// dA [K, r] = X^T (s G) from X [M, K] and ghlT [2r, pad8(M)];
+// dA [K, r] = scale_dA * X^T (s G) from X [M, K] (the adapter input: under dropout its
+// kept elements, with scale_dA = 1/(1-p)) and ghlT [2r, pad8(M)];
 // dB [r, N] = (s XA)^T dY from dY [M, N] and xahlT [2r, pad8(M)].
+// With `accumulate` both are added into dA and dB.
 qlora_status launch_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t K, int64_t N,
                           const uint16_t *ghlT, const uint16_t *xahlT, int r, float *dA, float *dB,
-                          int sms, cudaStream_t st) {
+                          int sms, cudaStream_t st, float scale_dA = 1.0f, int accumulate = 0) {
   LoraMmaParams p{};
   p.grad = 1;
+  p.out_scale = scale_dA;
+  p.out_scale1 = 1.0f;
+  p.accumulate = accumulate;
   p.r = r;
   p.out = dA;
   p.layout = 0;
@@ -465,6 +478,13 @@ qlora_status launch_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int6
   const LmOperands a{X, M, K, ghlT, 2 * r, M, pad8(M), K};
   const LmOperands b{dY, M, N, xahlT, 2 * r, M, pad8(M), N};
   return launch_lora_mma<true>(a, M, 2 * r, p, sms, st, &b);
+}
+
+// Xd = X (.) keep (bit-packed mask), n = M K elements, a multiple of 8.
+qlora_status launch_mask(const uint16_t *X, const uint8_t *keep, int64_t n, uint16_t *Xd, int sms, cudaStream_t st) {
+  LaunchTimer lt(QLORA_K_PREP, st);
+  mask_input_kernel<<<grid_for(n / 8, sms), 256, 0, st>>>(X, keep, n / 8, Xd);
+  return cuda_status(cudaGetLastError());
 }
 
 qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT, int sms, cudaStream_t st) {
@@ -508,14 +528,17 @@ bool skinny_launchable(const SkinnyPlan &pl, int64_t N) {
   return n > 0;
 }
 
+// xa_src is the adapter input (X, or X (.) keep under dropout) and xa_scale the factor of
+// its product (1, or 1/(1-p)).
 qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, const uint16_t *A,
                            const uint16_t *B, int r, float s, uint16_t *Y, float *xa,
-                           const SkinnyPlan &pl, cudaStream_t st) {
+                           const SkinnyPlan &pl, cudaStream_t st, const uint16_t *xa_src, float xa_scale) {
   const int64_t N = Wq->rows, K = Wq->cols;
   // 1. XA = X A by one cluster; it lets the dependent launch below start at once
   {
     XaParams xp{};
-    xp.X = X;
+    xp.X = xa_src;
+    xp.scale = xa_scale;
     xp.A = A;
     xp.xa = xa;
     xp.M = static_cast<int>(M);
@@ -596,10 +619,13 @@ qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, 
 
 // One fused GEMM launch.  MODE fwd: Y = X deq(W)^T + LoRA; MODE dx: dX = dY deq(W) + LoRA.
 // `sp` is the launch's split scratch, its counters already cleared in stream order.
+// keep (dX only, may be null): the bit-packed dropout mask of the adapter input, with
+// keep_scale = 1/(1-p).
 template <int MODE>
 qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
                          const uint16_t *lora_act_hl, const uint16_t *lora_w, int r,
-                         uint16_t *out, const SplitScratch &sp, int sms, cudaStream_t st) {
+                         uint16_t *out, const SplitScratch &sp, int sms, cudaStream_t st,
+                         const uint8_t *keep = nullptr, float keep_scale = 1.0f) {
   const int64_t N = Wq->rows, K = Wq->cols;
   const int64_t contraction = (MODE == kModeFwd) ? K : N;
   CUtensorMap tm_act, tm_codes, tm_lora;
@@ -645,9 +671,130 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
   p.kb_mid = p.kb_main / 2;
   p.scratch = sp.partial;
   p.flags = sp.flags;
+  p.keep32 = (MODE == kModeDx) ? reinterpret_cast<const uint32_t *>(keep) : nullptr;
+  p.keep_scale = keep_scale;
   LaunchTimer lt(MODE == kModeFwd ? QLORA_K_GEMM_FWD : QLORA_K_GEMM_DX, st);
   qlora_gemm_kernel<MODE><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_lora, p);
   return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------------------ the linear layer
+// keep (nullable): bit-packed keep mask of the adapter input X [M, K] (element m K + k
+// in bit (m K + k) mod 8 of byte (m K + k) / 8); kept values are scaled by 1/(1-p).
+qlora_status check_dropout(const uint8_t *keep, float p) {
+  if (!keep) return QLORA_OK;
+  if (!(p >= 0.0f && p < 1.0f)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(keep)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+size_t mask_workspace(int64_t M, int64_t K) { return align256(static_cast<size_t>(M) * K * 2); }
+
+qlora_status linear_fwd_impl(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, const uint16_t *A,
+                             const uint16_t *B, int r, float s, const uint8_t *keep, float drop_p,
+                             uint16_t *Y, float *XA_out, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  qlora_status st = check_nf4(Wq);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
+      (XA_out && !aligned16(XA_out)) || (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  if (!(s == s)) return QLORA_ERR_INVALID_ARG;
+  if ((st = check_dropout(keep, drop_p)) != QLORA_OK) return st;
+  DeviceInfo *d = nullptr;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t N = Wq->rows, K = Wq->cols;
+  const size_t need = fwd_workspace(M, N, K, r, d->sms) + (keep ? mask_workspace(M, K) : 0);
+  if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
+  Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
+  // the adapter input: X, or X (.) keep under dropout (its products then carry 1/(1-p))
+  const uint16_t *xin = X;
+  const float xscale = keep ? 1.0f / (1.0f - drop_p) : 1.0f;
+  if (keep) {
+    uint16_t *Xd = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * K * 2));
+    if (!Xd) return QLORA_ERR_WORKSPACE;
+    if ((st = launch_mask(X, keep, M * K, Xd, d->sms, stream)) != QLORA_OK) return st;
+    xin = Xd;
+  }
+  if (M <= kSkinnyMaxTokens) {
+    SkinnyPlan pl{};
+    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) {
+      float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
+      if (!xa) return QLORA_ERR_WORKSPACE;
+      return launch_skinny(X, M, Wq, A, B, r, s, Y, xa, pl, stream, xin, xscale);
+    }
+  }
+  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
+  uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
+  float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
+  SplitScratch sp;
+  if (!AT || !hl || !xa || !take_split(ws, gemm_split(M, N, K, d->sms), sp)) return QLORA_ERR_WORKSPACE;
+  // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps;
+  // the projection also clears the GEMM's split counters
+  if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+  if ((st = launch_projection(xin, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream, &sp, xscale)) != QLORA_OK)
+    return st;
+  return launch_gemm<kModeFwd>(X, M, Wq, hl, B, r, Y, sp, d->sms, stream);
+}
+
+qlora_status linear_bwd_impl(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
+                             const qlora_nf4_t *Wq, const uint16_t *A, const uint16_t *B, int r, float s,
+                             const uint8_t *keep, float drop_p, int accumulate, uint16_t *dX, float *dA,
+                             float *dB, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  qlora_status st = check_nf4(Wq);
+  if (st != QLORA_OK) return st;
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+      !aligned16(dB) || (dX && !aligned16(dX)) || (XA && !aligned16(XA)) ||
+      (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  if (!(s == s)) return QLORA_ERR_INVALID_ARG;
+  if ((st = check_dropout(keep, drop_p)) != QLORA_OK) return st;
+  DeviceInfo *d = nullptr;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t N = Wq->rows, K = Wq->cols;
+  const size_t need = bwd_workspace(M, N, K, r, d->sms) + (keep ? mask_workspace(M, K) : 0);
+  if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
+  Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
+  const uint16_t *xin = X;
+  const float xscale = keep ? 1.0f / (1.0f - drop_p) : 1.0f;
+  if (keep) {
+    uint16_t *Xd = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * K * 2));
+    if (!Xd) return QLORA_ERR_WORKSPACE;
+    if ((st = launch_mask(X, keep, M * K, Xd, d->sms, stream)) != QLORA_OK) return st;
+    xin = Xd;
+  }
+  const size_t hlT_bytes = static_cast<size_t>(2 * r) * pad8(M) * 2;
+  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
+  float *G = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
+  uint16_t *ghl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
+  uint16_t *ghlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
+  uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
+  float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
+  SplitScratch sp;
+  if (!AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
+  if (dX && !take_split(ws, gemm_split(M, K, N, d->sms), sp)) return QLORA_ERR_WORKSPACE;
+  // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from the adapter input)
+  if (XA) {
+    if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
+  } else {
+    if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
+    if ((st = launch_projection(xin, M, K, AT, r, s, xa_ws, nullptr, xahlT, d->sms, stream, nullptr, xscale)) !=
+        QLORA_OK)
+      return st;
+  }
+  // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA); clears the dX GEMM's
+  // split counters
+  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream, &sp)) != QLORA_OK) return st;
+  if (dX) {
+    if ((st = launch_gemm<kModeDx>(dY, M, Wq, ghl, A, r, dX, sp, d->sms, stream, keep, xscale)) != QLORA_OK)
+      return st;
+  }
+  // dA = (1/(1-p)) X_kept^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
+  return launch_grads(xin, dY, M, K, N, ghlT, xahlT, r, dA, dB, d->sms, stream, xscale, accumulate);
 }
 
 }  // namespace
@@ -694,6 +841,19 @@ size_t qlora_nf4_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, size_t *
   if (q8_bytes) *q8_bytes = q;
   if (step_bytes) *step_bytes = s;
   return c + q + s;
+}
+
+size_t qlora_nf4_single_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, size_t *step_bytes) {
+  if (rows <= 0 || cols <= 0) {
+    if (codes_bytes) *codes_bytes = 0;
+    if (step_bytes) *step_bytes = 0;
+    return 0;
+  }
+  const uint64_t n = static_cast<uint64_t>(rows) * static_cast<uint64_t>(cols);
+  const size_t c = static_cast<size_t>((n + 1) / 2), s = static_cast<size_t>(4 * ((n + 63) / 64));
+  if (codes_bytes) *codes_bytes = c;
+  if (step_bytes) *step_bytes = s;
+  return c + s;
 }
 
 qlora_status qlora_nf4_quantize(const uint16_t *W, int64_t rows, int64_t cols,
@@ -754,89 +914,83 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
   return f > b ? f : b;
 }
 
+size_t qlora_linear_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  const size_t b = qlora_linear_workspace_bytes(M, N, K, r);
+  return b ? b + mask_workspace(M, K) : 0;
+}
+
 qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
                               const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y,
                               float *XA_out, void *workspace, size_t workspace_bytes,
                               qlora_stream_t stream) {
-  qlora_status st = check_nf4(Wq);
-  if (st != QLORA_OK) return st;
-  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
-  if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
-      (XA_out && !aligned16(XA_out)) || (workspace && !aligned16(workspace)))
-    return QLORA_ERR_MISALIGNED;
-  if (!(s == s)) return QLORA_ERR_INVALID_ARG;
-  DeviceInfo *d = nullptr;
-  if ((st = device_info(&d)) != QLORA_OK) return st;
-  const int64_t N = Wq->rows, K = Wq->cols;
-  if (!workspace || workspace_bytes < fwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
-  if (M <= kSkinnyMaxTokens) {
-    SkinnyPlan pl{};
-    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) {
-      Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
-      float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-      if (!xa) return QLORA_ERR_WORKSPACE;
-      return launch_skinny(X, M, Wq, A, B, r, s, Y, xa, pl, stream);
-    }
-  }
-  Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
-  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
-  uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
-  float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  SplitScratch sp;
-  if (!AT || !hl || !xa || !take_split(ws, gemm_split(M, N, K, d->sms), sp)) return QLORA_ERR_WORKSPACE;
-  // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps;
-  // the projection also clears the GEMM's split counters
-  if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-  if ((st = launch_projection(X, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream, &sp)) != QLORA_OK)
-    return st;
-  return launch_gemm<kModeFwd>(X, M, Wq, hl, B, r, Y, sp, d->sms, stream);
+  return linear_fwd_impl(X, M, Wq, A, B, r, s, nullptr, 0.0f, Y, XA_out, workspace, workspace_bytes, stream);
+}
+
+qlora_status qlora_linear_fwd_ex(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
+                                 const uint16_t *A, const uint16_t *B, int r, float s,
+                                 const uint8_t *keep, float dropout_p, uint16_t *Y, float *XA_out,
+                                 void *workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  return linear_fwd_impl(X, M, Wq, A, B, r, s, keep, dropout_p, Y, XA_out, workspace, workspace_bytes, stream);
 }
 
 qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
                               const qlora_nf4_t *Wq, const uint16_t *A, const uint16_t *B, int r,
                               float s, uint16_t *dX, float *dA, float *dB, void *workspace,
                               size_t workspace_bytes, qlora_stream_t stream) {
-  qlora_status st = check_nf4(Wq);
-  if (st != QLORA_OK) return st;
-  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
-  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
-      !aligned16(dB) || (dX && !aligned16(dX)) || (XA && !aligned16(XA)) ||
-      (workspace && !aligned16(workspace)))
+  return linear_bwd_impl(dY, X, XA, M, Wq, A, B, r, s, nullptr, 0.0f, 0, dX, dA, dB, workspace,
+                         workspace_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_ex(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
+                                 const qlora_nf4_t *Wq, const uint16_t *A, const uint16_t *B, int r,
+                                 float s, const uint8_t *keep, float dropout_p, int accumulate,
+                                 uint16_t *dX, float *dA, float *dB, void *workspace,
+                                 size_t workspace_bytes, qlora_stream_t stream) {
+  return linear_bwd_impl(dY, X, XA, M, Wq, A, B, r, s, keep, dropout_p, accumulate, dX, dA, dB, workspace,
+                         workspace_bytes, stream);
+}
+
+qlora_status qlora_nf4_merge(const qlora_nf4_t *Wq, const uint16_t *W16, int64_t N, int64_t K,
+                             const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *W_out,
+                             qlora_stream_t stream) {
+  if ((Wq == nullptr) == (W16 == nullptr) || !A || !B || !W_out) return QLORA_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || N > (1ll << 24) || K > (1ll << 24) || N * K > (1ll << 40)) return QLORA_ERR_INVALID_ARG;
+  if (r < 8 || r > 128 || (r % 8) != 0 || !(s == s)) return QLORA_ERR_INVALID_ARG;
+  if ((N % 8) != 0 || (K % 64) != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (Wq) {
+    const qlora_status st = check_nf4(Wq);
+    if (st != QLORA_OK) return st;
+    if (Wq->rows != N || Wq->cols != K) return QLORA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(A) || !aligned16(B) || !aligned16(W_out) || (W16 && !aligned16(W16)))
     return QLORA_ERR_MISALIGNED;
-  if (!(s == s)) return QLORA_ERR_INVALID_ARG;
   DeviceInfo *d = nullptr;
-  if ((st = device_info(&d)) != QLORA_OK) return st;
-  const int64_t N = Wq->rows, K = Wq->cols;
-  if (!workspace || workspace_bytes < bwd_workspace(M, N, K, r, d->sms)) return QLORA_ERR_WORKSPACE;
-  Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
-  const size_t hlT_bytes = static_cast<size_t>(2 * r) * pad8(M) * 2;
-  uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
-  float *G = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  uint16_t *ghl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
-  uint16_t *ghlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
-  uint16_t *xahlT = static_cast<uint16_t *>(ws.take(hlT_bytes));
-  float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
-  SplitScratch sp;
-  if (!AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
-  if (dX && !take_split(ws, gemm_split(M, K, N, d->sms), sp)) return QLORA_ERR_WORKSPACE;
-  // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from X and A)
-  if (XA) {
-    if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
-  } else {
-    if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
-    if ((st = launch_projection(X, M, K, AT, r, s, xa_ws, nullptr, xahlT, d->sms, stream)) != QLORA_OK)
-      return st;
+  qlora_status st = device_info(&d);
+  if (st != QLORA_OK) return st;
+  MergeParams p{};
+  if (Wq) {
+    p.codes = Wq->codes;
+    p.q8 = Wq->q8;
+    p.step = Wq->step;
   }
-  // G = dY B^T; s*G hi|lo in [M, 2r] (dX GEMM) and [2r, M] (dA); clears the dX GEMM's
-  // split counters
-  if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream, &sp)) != QLORA_OK) return st;
-  if (dX) {
-    if ((st = launch_gemm<kModeDx>(dY, M, Wq, ghl, A, r, dX, sp, d->sms, stream)) != QLORA_OK) return st;
-  }
-  // dA = X^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
-  return launch_grads(X, dY, M, K, N, ghlT, xahlT, r, dA, dB, d->sms, stream);
+  p.w16 = W16;
+  p.out = W_out;
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.stages = (r + 63) / 64;
+  p.s = s;
+  p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
+  std::memcpy(p.levels, nf4_tables().levels, sizeof(p.levels));
+  CUtensorMap tm_bt, tm_a;
+  // B [r, N]: x = n (inner), y = j; A [K, r]: x = j (inner), y = k.  Boxes reach j = 64 per
+  // stage; rows j >= r are outside the tensors and arrive as zeros.
+  if (!make_map_2d(&tm_bt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, r * 2, 64, kMgCols, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>((K + kMgCols - 1) / kMgCols), static_cast<unsigned>((N + kMgRows - 1) / kMgRows));
+  LaunchTimer lt(QLORA_K_MERGE, stream);
+  nf4_merge_kernel<<<grid, kMgThreads, merge_smem_bytes(p.stages), stream>>>(tm_bt, tm_a, p);
+  return cuda_status(cudaGetLastError());
 }
 
 qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags) {

@@ -273,9 +273,14 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
       }
     }
 
-    // second level: one constant per group (threads 0..255, one block each)
+    // second level: one constant per group (threads 0..255, one block each); with
+    // single-level constants (q8 null) the block absmax itself is stored in fp32
     const int64_t b = g * kGroup + tid;
     const float a = (tid < kGroup && b < nblocks) ? amax[tid] : 0.f;
+    if (q8 == nullptr) {
+      if (tid < kGroup && b < nblocks) step[b] = a;
+      continue;
+    }
     float m = a;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -298,7 +303,8 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
 }
 
 // Standalone dequant: 16 values per thread per iteration (8 bytes of codes in,
-// 32 bytes of bf16 out), grid-stride.  w = bf16_RN(RN32(L[code] * RN32(q8*step))).
+// 32 bytes of bf16 out), grid-stride.  w = bf16_RN(RN32(L[code] * RN32(q8*step))),
+// or bf16_RN(RN32(L[code] * step[b])) with single-level constants (q8 null).
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(
     const uint8_t *__restrict__ codes, const uint8_t *__restrict__ q8,
     const float *__restrict__ step, int64_t n, uint16_t *__restrict__ out,
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
     const int64_t e = u << 4;
     const uint2 c = *reinterpret_cast<const uint2 *>(codes + (e >> 1));
     const int64_t b = e >> 6;
-    const float sc = __fmul_rn(static_cast<float>(q8[b]), step[b >> 8]);
+    const float sc = q8 ? __fmul_rn(static_cast<float>(q8[b]), step[b >> 8]) : step[b];
     uint32_t o[8];
     const uint32_t cw[2] = {c.x, c.y};
 #pragma unroll
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
       const uint8_t byte = codes[e >> 1];
       const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 15u);
       const int64_t b = e >> 6;
-      const float sc = __fmul_rn(static_cast<float>(q8[b]), step[b >> 8]);
+      const float sc = q8 ? __fmul_rn(static_cast<float>(q8[b]), step[b >> 8]) : step[b];
       const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(L[code], sc));
       out[e] = *reinterpret_cast<const uint16_t *>(&h);
     }

@@ -45,7 +45,7 @@ constexpr int kSkPre = 4;          // macro-blocks of block constants prefetched
 struct SkinnyParams {
   const uint16_t *X;      // [M, K] bf16
   const uint8_t *codes;   // packed NF4 of W [N, K]
-  const uint8_t *q8;
+  const uint8_t *q8;      // null: single-level constants, step[block] = the block absmax
   const float *step;
   const uint16_t *B;      // [r, N] bf16
   const float *xa;        // [M, r] fp32, written by qlora_xa_kernel
@@ -142,10 +142,12 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
     qa[i] = qb[i] = 0u;
     sa[i] = sb[i] = 0.f;
     if (blk < nblk) {
-      qa[i] = p.q8[ba + blk];
-      qb[i] = p.q8[bb + blk];
-      sa[i] = p.step[(ba + blk) >> 8];
-      sb[i] = p.step[(bb + blk) >> 8];
+      // single-level constants (q8 null): code 1 and the block's own constant, so the
+      // scale RN32(1 * a_b) = a_b exactly
+      qa[i] = p.q8 ? p.q8[ba + blk] : 1u;
+      qb[i] = p.q8 ? p.q8[bb + blk] : 1u;
+      sa[i] = p.q8 ? p.step[(ba + blk) >> 8] : p.step[ba + blk];
+      sb[i] = p.q8 ? p.step[(bb + blk) >> 8] : p.step[bb + blk];
     }
   }
   float L[16];
@@ -172,10 +174,10 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
       qa[kSkPre - 1] = qb[kSkPre - 1] = 0u;
       sa[kSkPre - 1] = sb[kSkPre - 1] = 0.f;
       if (blk < nblk) {
-        qa[kSkPre - 1] = p.q8[ba + blk];
-        qb[kSkPre - 1] = p.q8[bb + blk];
-        sa[kSkPre - 1] = p.step[(ba + blk) >> 8];
-        sb[kSkPre - 1] = p.step[(bb + blk) >> 8];
+        qa[kSkPre - 1] = p.q8 ? p.q8[ba + blk] : 1u;
+        qb[kSkPre - 1] = p.q8 ? p.q8[bb + blk] : 1u;
+        sa[kSkPre - 1] = p.q8 ? p.step[(ba + blk) >> 8] : p.step[ba + blk];
+        sb[kSkPre - 1] = p.q8 ? p.step[(bb + blk) >> 8] : p.step[bb + blk];
       }
     }
     ok = __all_sync(0xffffffffu, wait_bar(&bars[mb], 0, waiter));
@@ -272,12 +274,13 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
 constexpr int kXaCluster = 8;
 
 struct XaParams {
-  const uint16_t *X;   // [M, K] bf16
+  const uint16_t *X;   // [M, K] bf16 (the adapter input: dropped-out elements already zero)
   const uint16_t *A;   // [K, r] bf16
   float *xa;           // [M, r] fp32
   int M, K, r, kx;
   int chunk;           // contraction rows per pass, a multiple of 16
   uint64_t limit_ns;
+  float scale;         // applied to the sum before it is stored (1/(1-p) under dropout)
 };
 
 inline int xa_chunk_rows(int r) { return r <= 64 ? 512 : 256; }
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(256, 1) qlora_xa_kernel(const __grid_constant_
       float v = 0.f;
 #pragma unroll
       for (int q = 0; q < kXaCluster; ++q) v += ld_dsmem_f32(map_rank(base + 4u * i, q));
-      p.xa[i] = v;
+      p.xa[i] = __fmul_rn(v, p.scale);
     }
   }
   cluster_sync_all();   // the peers' partials stay until rank 0 has read them

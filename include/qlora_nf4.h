@@ -70,6 +70,10 @@ typedef enum {
  *   q8    : ceil(n/64) bytes, the 8-bit code of each block's absmax constant.
  *   step  : ceil(n/16384) floats, the fp32 second-level constant of each group;
  *           block b's constant is reconstructed as RN32(q8[b] * step[b/256]).
+ * Single-level constants ([STEPS] Step 2 without Step 3: one 32-bit constant per
+ * block, half a bit per value): q8 = NULL and step holds ceil(n/64) floats, block
+ * b's absmax itself (4.5 bits per value in all).  Every entry point that takes a
+ * qlora_nf4_t accepts either form; quantize writes the form its `out` names.
  */
 typedef struct {
   uint8_t *codes;
@@ -102,6 +106,9 @@ void qlora_nf4_levels(float out[16]);
 size_t qlora_nf4_bytes(int64_t rows, int64_t cols, size_t *codes_bytes,
                        size_t *q8_bytes, size_t *step_bytes);
 
+/* Byte sizes for single-level constants: codes as above, 4*ceil(n/64) of step. */
+size_t qlora_nf4_single_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, size_t *step_bytes);
+
 /*
  * Quantize a bf16 weight W[rows, cols] ([STEPS] Steps 1-3, [NF4]).
  *   a_b  = max |w| over each 64-value block (the last block may be partial);
@@ -109,6 +116,7 @@ size_t qlora_nf4_bytes(int64_t rows, int64_t cols, size_t *codes_bytes,
  *          the zero level);
  *   c_g  = max a_b over each group of 256 blocks; step_g = RN32(c_g / 255);
  *   q8_b = min(255, round_half_even(RN32(a_b / step_g)))   (0 when c_g = 0).
+ * With out->q8 = NULL (single-level constants) step[b] = a_b instead.
  * Any n = rows*cols >= 1.  `out` is a host struct whose arrays (sized by
  * qlora_nf4_bytes) receive the result; rows/cols in `out` must equal the
  * arguments.  Non-finite input values give unspecified codes and set
@@ -119,7 +127,8 @@ qlora_status qlora_nf4_quantize(const uint16_t *W, int64_t rows, int64_t cols,
 
 /*
  * Dequantize to bf16 ([STEPS] "A worked example" 4; [SPLIT]):
- *   W_out[i] = bf16_RN( RN32( L[code_i] * RN32(q8[b] * step[b/256]) ) ).
+ *   W_out[i] = bf16_RN( RN32( L[code_i] * RN32(q8[b] * step[b/256]) ) ),
+ * or bf16_RN( RN32( L[code_i] * step[b] ) ) with single-level constants.
  * W_out holds rows*cols bf16 values.
  */
 qlora_status qlora_nf4_dequant(const qlora_nf4_t *Wq, uint16_t *W_out,
@@ -155,6 +164,28 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *W
                               const uint16_t *A, const uint16_t *B, int r, float s,
                               uint16_t *Y, float *XA_out, void *workspace,
                               size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * Forward with dropout on the adapter input ("QLoRA", ozercemkelahmet.com, "A code
+ * example with common libraries": lora_dropout), otherwise as qlora_linear_fwd:
+ *   Xd = X (.) keep / (1 - p)     (inverted dropout; the frozen path sees X itself)
+ *   XA = Xd A                     (fp32 [M, r])
+ *   Y  = X deq(W)^T + s * XA B
+ * keep: device, bit-packed mask of X [M, K] drawn by the caller (Bernoulli(1 - p)
+ * per element): element m K + k is kept when bit (m K + k) mod 8 of byte
+ * (m K + k) / 8 is set; 16-byte aligned; M*K/8 bytes.  NULL: no dropout (p is then
+ * ignored).  p in [0, 1).  X (.) keep is formed exactly (a zeroing) in the
+ * workspace, whose size is then qlora_linear_dropout_workspace_bytes; the fp32
+ * product is multiplied by 1/(1-p) before it is stored.
+ */
+qlora_status qlora_linear_fwd_ex(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq,
+                                 const uint16_t *A, const uint16_t *B, int r, float s,
+                                 const uint8_t *keep, float dropout_p, uint16_t *Y, float *XA_out,
+                                 void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Workspace bytes of the _ex calls with a dropout mask: the plain size plus room for
+ * X (.) keep (M*K bf16). */
+size_t qlora_linear_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Forward without a workspace argument, for callers that cannot allocate device
@@ -203,6 +234,41 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
                               size_t workspace_bytes, qlora_stream_t stream);
 
 /*
+ * The adapter folded into a 16-bit weight for serving ("QLoRA", ozercemkelahmet.com,
+ * How it works, Step 8 and section "Merging after QLoRA"):
+ *   W_out[n][k] = bf16_RN( base[n][k] + s * sum_j B[j][n] A[k][j] )
+ * base is the bf16 original W16 [N, K] (the page's preferred route) or the
+ * dequantized NF4 weight Wq (exactly the element qlora_nf4_dequant gives); pass
+ * exactly one of them.  The sum s*(A B)^T + base is formed with one fp32 FMA per
+ * element (the rank-r product accumulated in fp32 on the tensor cores) and rounded
+ * once to bf16.  N a multiple of 8, K of 64; r in [8, 128], a multiple of 8.
+ * W_out [N, K] bf16 must not overlap the inputs.
+ */
+qlora_status qlora_nf4_merge(const qlora_nf4_t *Wq, const uint16_t *W16, int64_t N, int64_t K,
+                             const uint16_t *A, const uint16_t *B, int r, float s,
+                             uint16_t *W_out, qlora_stream_t stream);
+
+/*
+ * Backward with adapter-input dropout and gradient accumulation ("QLoRA",
+ * ozercemkelahmet.com, "A code example with common libraries": lora_dropout;
+ * "Training arguments": gradient_accumulation_steps), otherwise as
+ * qlora_linear_bwd.  With the forward's mask (same keep, same p):
+ *   G  = dY B^T
+ *   dX = dY deq(W) + s * (G A^T) (.) keep / (1 - p)   (one bf16 rounding)
+ *   dA = s * Xd^T G,  Xd = X (.) keep / (1 - p)
+ *   dB = s * XA^T dY  (XA from qlora_linear_fwd_ex, or recomputed from Xd if NULL)
+ * accumulate != 0 adds the results into dA and dB instead of overwriting them (the
+ * micro-batches of one optimizer step).  keep, p and the workspace as in
+ * qlora_linear_fwd_ex; keep = NULL: no dropout.
+ */
+qlora_status qlora_linear_bwd_ex(const uint16_t *dY, const uint16_t *X, const float *XA,
+                                 int64_t M, const qlora_nf4_t *Wq, const uint16_t *A,
+                                 const uint16_t *B, int r, float s, const uint8_t *keep,
+                                 float dropout_p, int accumulate, uint16_t *dX, float *dA,
+                                 float *dB, void *workspace, size_t workspace_bytes,
+                                 qlora_stream_t stream);
+
+/*
  * Synchronizes `stream`, then returns the device status word of the current
  * device in *flags (QLORA_DEVSTAT_* bits) and clears it.  Returns
  * QLORA_ERR_TIMEOUT / QLORA_ERR_DEVICE_CHECK when the corresponding bit was set.
@@ -242,7 +308,8 @@ typedef enum {
   QLORA_K_GEMM_DX = 5,      /* fused dequant GEMM, dX               */
   QLORA_K_GRAD = 6,         /* adapter gradients dA and dB (one     */
                             /* launch computes both)                */
-  QLORA_K_SKINNY = 7        /* few-token forward                    */
+  QLORA_K_SKINNY = 7,       /* few-token forward                    */
+  QLORA_K_MERGE = 8         /* adapter merged into a 16-bit weight  */
 } qlora_kernel_kind;
 
 qlora_status qlora_profile_enable(int on);

@@ -26,6 +26,7 @@ from .generators import (  # noqa: F401
     normal_bf16,
     normal_bf16_rows,
     heavy_tail_chunk,
+    keep_mask,
     CHUNK_ELEMS,
     n_chunks,
     linear_problem,

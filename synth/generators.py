@@ -83,6 +83,13 @@ def linear_problem_rows(M: int, N: int, K: int, r: int, alpha: float, w_std: flo
     return LinearProblem(tag + f"[:{tokens}]", tokens, N, K, r, alpha, W, X, A, B, dY)
 
 
+def keep_mask(seed: int, tag: str, shape, p: float) -> np.ndarray:
+    """A dropout keep mask: True with probability 1 - p per element, independently
+    (drawn as uniform fp32 < 1 - p)."""
+    g = np.random.default_rng([seed, _tag_id("keep" + tag), 0])
+    return g.random(shape, dtype=np.float32) < np.float32(1.0 - p)
+
+
 def n_chunks(n: int) -> int:
     return (n + CHUNK_ELEMS - 1) // CHUNK_ELEMS
 

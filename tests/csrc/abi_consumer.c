@@ -46,6 +46,9 @@ int main(void) {
   CHECK(cb == 8388608u && qb == 262144u && sb == 4096u);
   CHECK(qlora_nf4_bytes(1, 65, &cb, &qb, &sb) == 33u + 2u + 4u);
   CHECK(qlora_nf4_bytes(3, 5, NULL, NULL, NULL) == 8u + 1u + 4u);
+  /* single-level constants: one fp32 per 64-value block */
+  CHECK(qlora_nf4_single_bytes(4096, 4096, &cb, &sb) == 8388608u + 4u * 262144u);
+  CHECK(qlora_nf4_single_bytes(1, 65, NULL, NULL) == 33u + 8u);
 
   /* workspace: positive for a valid call, 0 for an invalid one */
   CHECK(qlora_linear_workspace_bytes(4096, 4096, 4096, 16) > 0);
@@ -76,6 +79,17 @@ int main(void) {
                          NULL) == QLORA_ERR_INVALID_ARG);
   CHECK(qlora_linear_bwd(NULL, PTR(16), NULL, 4, &w, PTR(16), PTR(16), 8, 1.0f, NULL, PTR(16), PTR(16),
                          PTR(16), 1u << 20, NULL) == QLORA_ERR_INVALID_ARG);
+  /* merge: exactly one base, r a multiple of 8 in [8, 128], N % 8 == 0, K % 64 == 0 */
+  CHECK(qlora_nf4_merge(NULL, NULL, 128, 128, PTR(16), PTR(16), 16, 1.0f, PTR(16), NULL) ==
+        QLORA_ERR_INVALID_ARG);
+  CHECK(qlora_nf4_merge(&w, PTR(16), 128, 128, PTR(16), PTR(16), 16, 1.0f, PTR(16), NULL) ==
+        QLORA_ERR_INVALID_ARG);
+  CHECK(qlora_nf4_merge(NULL, PTR(16), 128, 128, PTR(16), PTR(16), 12, 1.0f, PTR(16), NULL) ==
+        QLORA_ERR_INVALID_ARG);
+  CHECK(qlora_nf4_merge(NULL, PTR(16), 100, 128, PTR(16), PTR(16), 16, 1.0f, PTR(16), NULL) ==
+        QLORA_ERR_UNSUPPORTED_SHAPE);
+  CHECK(qlora_nf4_merge(NULL, PTR(16), 128, 128, PTR(16), PTR(16), 16, 1.0f, PTR(24), NULL) ==
+        QLORA_ERR_MISALIGNED);
   CHECK(qlora_selftest_wait_timeout(0, NULL) == QLORA_ERR_INVALID_ARG);
   CHECK(qlora_get_device_status(NULL, NULL) == QLORA_ERR_INVALID_ARG);
   CHECK(qlora_profile_read(0, NULL, NULL) == 0);   /* nothing recorded: profiling never enabled */

@@ -57,3 +57,20 @@ def test_row_prefix_generators_match_the_full_tensors():
     s = linear_problem_rows(40, 96, 128, 8, 16.0, 0.02, 7, 33, seed=2)
     assert np.array_equal(s.W, p.W[:33]) and np.array_equal(s.X, p.X[:7])
     assert np.array_equal(s.dY, p.dY[:7]) and np.array_equal(s.A, p.A) and np.array_equal(s.B, p.B)
+
+
+def test_keep_mask_rate_and_packing():
+    """keep_mask keeps each element with probability 1 - p; the binding's packer
+    (bit-packed, element i in bit i mod 8 of byte i / 8) agrees with numpy's."""
+    import torch
+    from synth import keep_mask
+    from bit_nf4_quantized_19_b200.api import pack_keep_mask
+    k = keep_mask(0, "rate", (1000, 1024), 0.1)
+    assert abs(k.mean() - 0.9) < 0.002
+    assert not np.array_equal(k, keep_mask(1, "rate", (1000, 1024), 0.1))
+    assert np.array_equal(k, keep_mask(0, "rate", (1000, 1024), 0.1))
+    got = pack_keep_mask(torch.from_numpy(k[:37, :64])).numpy()
+    assert np.array_equal(got, np.packbits(k[:37, :64].astype(np.uint8).ravel(), bitorder="little"))
+    e = np.zeros((1, 8), bool)
+    e[0, 3] = True
+    assert pack_keep_mask(torch.from_numpy(e)).tolist() == [8]
