@@ -18,12 +18,12 @@
 //   warp 0        TMA producer of the activation tiles (X / dY, or the LoRA
 //                 hi/lo operand).
 //   warp 1        TMEM allocator and single-thread MMA issuer.
-//   warp 2        weight producer: lane 0 TMA-loads the packed 4-bit codes of
-//                 each stage into their own ring (so the small weight stream runs
-//                 ahead of the activation ring instead of waiting behind it); all
-//                 32 lanes rebuild the stage's 128 block constants
-//                 RN32(q8 * step) from the 8-bit codes and the fp32 group
-//                 constants (read one stage ahead) next to them.
+//   warps 2, 3    weight producers, alternate stages: lane 0 TMA-loads the
+//                 packed 4-bit codes of a stage into their own ring (so the small
+//                 weight stream runs ahead of the activation ring instead of
+//                 waiting behind it); all 32 lanes rebuild the stage's 128 block
+//                 constants RN32(q8 * step) from the 8-bit codes and the fp32
+//                 group constants (requested one own stage ahead) next to them.
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
 //   warps 8..15   dequant producers, two warpgroups taking alternate stages:
 //                 packed codes + block constant -> bf16 tile in the
@@ -67,10 +67,6 @@ constexpr int kBStageBytes = kBN * 128;   // 32 KB
 constexpr int kAStageBytes = kWT * 128;   // 16 KB
 constexpr int kWStageBytes = 4096;        // packed codes of one stage
 constexpr int kSStageBytes = 512;         // 128 fp32 block constants of one stage
-#ifndef QLORA_GEMM_SCALE_PRE
-#define QLORA_GEMM_SCALE_PRE 6
-#endif
-constexpr int kScalePre = QLORA_GEMM_SCALE_PRE;   // stages of block constants requested ahead
 constexpr uint32_t kSplitArrive = 1u;     // split-tile counter: one per arriving half
 constexpr uint32_t kSplitReady = 16u;     // added once the first half's partial is stored
 constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
@@ -80,6 +76,7 @@ constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStagesB * kBStageBytes +
                                1024 /*barriers, flags, levels*/;
 static_assert(kGemmSmemBytes <= 227 * 1024, "GEMM shared memory exceeds the per-CTA limit");
 static_assert(kStagesW <= 32 && kStagesB <= 32, "ring bookkeeping uses 32-bit masks");
+static_assert(kStagesW % 2 == 0, "the two weight producer warps each keep to the slots of one parity");
 
 enum GemmMode : int { kModeFwd = 0, kModeDx = 1 };
 
@@ -150,27 +147,70 @@ QDEV uint32_t atom_acq_rel_add_u32(unsigned int *a, uint32_t v) {
   return old;
 }
 
-// The 128 block constants of one weight stage, RN32(q8 * step) for stage slot idx =
-// lane + 32 i:  fwd: weight row w0 + idx, block kb;  dX: weight row kb*64 + (idx & 63),
-// block w0/64 + (idx >> 6).  Raw values are loaded here and multiplied when stored.
+// One weight producer warp's walk over the W stages it owns (global W stage
+// counter c = c0 + j with c mod 2 = wp), with the block indices of its lane's four
+// constants kept incrementally: slot idx = lane + 32 i holds
+//   fwd: weight row w0 + idx, block kb;
+//   dX:  weight row kb*64 + (idx & 63), block w0/64 + (idx >> 6).
 template <int MODE>
-QDEV void load_stage_scales(const GemmParams &p, int w0, int kb, int lane, uint32_t (&q)[4], float (&st)[4]) {
+struct WStageCursor {
+  bool have;
+  int it, kb0, n, j, w0;
+  uint32_t c0;          // global W stage counter at the item's first stage
+  int64_t b[4];         // block index of the item's first stage
+  int64_t inc;          // block index step from one stage to the next
+
+  QDEV void enter(const GemmParams &p, int num_tiles, int lane) {
+    GemmItem w;
+    have = gemm_item(p, num_tiles, it, w);
+    if (!have) return;
+    kb0 = w.kb0;
+    n = w.kb1 - w.kb0;
+    w0 = (w.tile % p.num_w_tiles) * kWT;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int idx = lane + 32 * i;
-    int64_t b;
-    if (MODE == kModeFwd) b = static_cast<int64_t>(w0 + idx) * p.KB + kb;
-    else b = static_cast<int64_t>(kb * kBK + (idx & 63)) * p.KB + (w0 >> 6) + (idx >> 6);
-    if (p.q8) {
-      q[i] = __ldg(p.q8 + b);
-      st[i] = __ldg(p.step + (b >> 8));
-    } else {
-      // single-level constants: the block's own fp32 absmax, and RN32(1 * a_b) = a_b
-      q[i] = 1u;
-      st[i] = __ldg(p.step + b);
+    for (int i = 0; i < 4; ++i) {
+      const int idx = lane + 32 * i;
+      if (MODE == kModeFwd) b[i] = static_cast<int64_t>(w0 + idx) * p.KB + kb0;
+      else b[i] = static_cast<int64_t>(kb0 * kBK + (idx & 63)) * p.KB + (w0 >> 6) + (idx >> 6);
+    }
+    inc = (MODE == kModeFwd) ? 1 : static_cast<int64_t>(kBK) * p.KB;
+  }
+  // moves past the ends of items until stage j lies inside one (or none is left)
+  QDEV void settle(const GemmParams &p, int num_tiles, int lane) {
+    while (have && j >= n) {
+      j -= n;
+      c0 += static_cast<uint32_t>(n);
+      ++it;
+      enter(p, num_tiles, lane);
     }
   }
-}
+  QDEV void start(const GemmParams &p, int num_tiles, int lane, uint32_t wp) {
+    it = 0;
+    c0 = 0;
+    j = static_cast<int>(wp);
+    enter(p, num_tiles, lane);
+    settle(p, num_tiles, lane);
+  }
+  QDEV void advance(const GemmParams &p, int num_tiles, int lane) {
+    j += 2;
+    settle(p, num_tiles, lane);
+  }
+  // raw constants of stage j: (q8, step) or, single-level, (1, the block's absmax)
+  QDEV void load(const GemmParams &p, uint32_t (&q)[4], float (&st)[4]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t bi = b[i] + static_cast<int64_t>(j) * inc;
+      if (p.q8) {
+        q[i] = __ldg(p.q8 + bi);
+        st[i] = __ldg(p.step + (bi >> 8));
+      } else {
+        q[i] = 1u;
+        st[i] = __ldg(p.step + bi);
+      }
+    }
+  }
+};
+
 QDEV void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int MODE>
@@ -188,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float *sS = reinterpret_cast<float *>(sW + kStagesW * kWStageBytes);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sS + kStagesW * (kSStageBytes / 4));
   uint64_t *full_B = bars;                  // activation tile landed (TMA)
-  uint64_t *full_A = full_B + kStagesB;     // dequantized tile written (4 warp arrivals)
+  uint64_t *full_A = full_B + kStagesB;     // dequantized tile written (128 thread arrivals)
   uint64_t *empty_A = full_A + kStagesA;    // MMAs of the stage done: both tiles free
   uint64_t *full_W = empty_A + kStagesA;
   uint64_t *empty_W = full_W + kStagesW;
@@ -205,13 +245,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = tid & 31;
 
   if (tid == 0) {
+    // full_A: one arrival per dequant thread, each after its own stores and proxy fence
     for (int i = 0; i < kStagesA; ++i) {
       mbar_init(&full_B[i], 1);
-      mbar_init(&full_A[i], 4);
+      mbar_init(&full_A[i], 128);
       mbar_init(&empty_A[i], 1);
     }
-    // full_W: the TMA's expect_tx arrival plus one per lane of the weight producer
-    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 33); mbar_init(&empty_W[i], 4); }
+    // full_W: the TMA's expect_tx arrival plus one per lane of the weight producer;
+    // empty_W: one per consumer thread, each once it has used what it read
+    for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 33); mbar_init(&empty_W[i], 128); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -264,77 +306,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int s = 0; s < kStagesB; ++s)
         if (armedB & (1u << s)) wait_bar(&full_B[s], (lastB >> s) & 1u, final_wt);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ weight producer
-    // The raw constants of a stage are requested kScalePre stages before it is
-    // produced (a lookahead iterator runs that far ahead of the ring), so their L2
-    // latency stays off the producer's path.
-    int ws = 0;
-    uint32_t wph = 0;
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ weight producers
+    // Warp 2 takes the even W stages, warp 3 the odd ones (the W ring has an even
+    // number of slots, so each warp keeps to its own slots).  Per stage, lane 0
+    // TMA-loads the packed codes and all 32 lanes rebuild the 128 block constants;
+    // the raw constants of a warp's next stage are requested before it waits for the
+    // current one.
+    const uint32_t wp = static_cast<uint32_t>(warp - 2);
+    WStageCursor<MODE> cur;
+    cur.start(p, num_tiles, lane, wp);
+    uint32_t qc[4] = {0u, 0u, 0u, 0u}, qn[4] = {0u, 0u, 0u, 0u};
+    float sc[4] = {0.f, 0.f, 0.f, 0.f}, sn[4] = {0.f, 0.f, 0.f, 0.f};
+    if (cur.have) cur.load(p, qc, sc);
     uint32_t armedW = 0, lastW = 0;
-    GemmItem w, wa;
-    int it = 0, ita = 0;
-    bool have = gemm_item(p, num_tiles, 0, w);
-    int kb = have ? w.kb0 : 0;
-    bool have_a = have;
-    wa = w;
-    int kba = kb;
-    auto advance_a = [&]() {
-      if (!have_a) return;
-      if (++kba >= wa.kb1) {
-        ++ita;
-        have_a = gemm_item(p, num_tiles, ita, wa);
-        kba = have_a ? wa.kb0 : 0;
-      }
-    };
-    uint32_t qv[kScalePre][4];
-    float sv[kScalePre][4];
-#pragma unroll
-    for (int d = 0; d < kScalePre; ++d) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { qv[d][i] = 0u; sv[d][i] = 0.f; }
-      if (have_a) load_stage_scales<MODE>(p, (wa.tile % p.num_w_tiles) * kWT, kba, lane, qv[d], sv[d]);
-      advance_a();
-    }
-    while (have) {
-      const int w0 = (w.tile % p.num_w_tiles) * kWT;
+    while (cur.have) {
+      WStageCursor<MODE> nx = cur;
+      nx.advance(p, num_tiles, lane);
+      if (nx.have) nx.load(p, qn, sn);
+      const uint32_t c = cur.c0 + static_cast<uint32_t>(cur.j);
+      const int ws = static_cast<int>(c % kStagesW);
+      const uint32_t wph = (c / kStagesW) & 1u;
       // warp-uniform: every lane arrives on full_W below
       if (!__all_sync(0xffffffffu, wait_bar(&empty_W[ws], wph ^ 1u, wt))) break;
       if (lane == 0) {
+        const int kb = cur.kb0 + cur.j;
+        // the slot's previous codes were read through the generic proxy; the TMA
+        // below rewrites them through the async proxy: order the two
+        fence_proxy_async_smem();
         mbar_arrive_expect_tx(&full_W[ws], kWStageBytes);
         if (MODE == kModeFwd) {
           // codes: 32 bytes (64 values of K) x 128 weight rows
-          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, w0);
+          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], kb * 32, cur.w0);
         } else {
           // codes: 64 bytes (128 values of K from w0) x 64 weight rows n = kb*64..
-          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], w0 / 2, kb * kBK);
+          tma_load_2d(sW + ws * kWStageBytes, &tm_codes, &full_W[ws], cur.w0 / 2, kb * kBK);
         }
         armedW |= 1u << ws;
         lastW = (lastW & ~(1u << ws)) | (wph << ws);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        sS[ws * 128 + lane + 32 * i] = __fmul_rn(static_cast<float>(qv[0][i]), sv[0][i]);
+        sS[ws * 128 + lane + 32 * i] = __fmul_rn(static_cast<float>(qc[i]), sc[i]);
       mbar_arrive(&full_W[ws]);
-      if (++ws == kStagesW) { ws = 0; wph ^= 1u; }
-      // shift the prefetch ring and request the stage kScalePre ahead
+      cur = nx;
 #pragma unroll
-      for (int d = 0; d + 1 < kScalePre; ++d) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { qv[d][i] = qv[d + 1][i]; sv[d][i] = sv[d + 1][i]; }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { qv[kScalePre - 1][i] = 0u; sv[kScalePre - 1][i] = 0.f; }
-      if (have_a)
-        load_stage_scales<MODE>(p, (wa.tile % p.num_w_tiles) * kWT, kba, lane, qv[kScalePre - 1],
-                                sv[kScalePre - 1]);
-      advance_a();
-      // next stage
-      if (++kb >= w.kb1) {
-        ++it;
-        have = gemm_item(p, num_tiles, it, w);
-        kb = have ? w.kb0 : 0;
-      }
+      for (int i = 0; i < 4; ++i) { qc[i] = qn[i]; sc[i] = sn[i]; }
     }
     if (lane == 0) {
       volatile int no_abort = 0;
@@ -540,8 +557,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (main) {
           const int ws = static_cast<int>(my_w % kStagesW);
           const uint32_t wph = (my_w / kStagesW) & 1u;
-          // warp-uniform: the per-warp arrivals below need every lane on the same path
-          const bool w_ok = wait_bar(&full_W[ws], wph, wt) && wait_bar(&empty_A[as], aph ^ 1u, wt);
+          // warp-uniform: the per-warp arrivals below need every lane on the same path.
+          // The A slot first: once it is free the MMA has consumed A stage a_cnt - 4,
+          // so the dequant of W stage my_w - 6 (an earlier stage, whichever warpgroup
+          // took it) has passed its own wait on this W slot, whose barrier is then at
+          // least in the phase this wait names.  (Waiting on full_W first could see a
+          // phase two behind and take the previous parity's completion for this one.)
+          const bool w_ok = wait_bar(&empty_A[as], aph ^ 1u, wt) && wait_bar(&full_W[ws], wph, wt);
           if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
           uint32_t src, dst;
           int swz;
@@ -563,8 +585,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint4 c0 = ld_shared_v4(src);
           const uint4 c1 = ld_shared_v4(src + 16);
-          __syncwarp();                     // the warp's codes are in registers now
-          if (lane == 0) mbar_arrive(&empty_W[ws]);
           Nf4Lut lut;
           nf4_build_lut(L, sc, lut);
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -574,9 +594,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             nf4_decode8(cw[c], lut, o);
             st_shared_v4(dst + ((c ^ swz) << 4), o[0], o[1], o[2], o[3]);
           }
+          // the W slot is released by every thread itself, and only once the decode
+          // above has used the codes and the constant it read: the producer then
+          // rewrites the constants and (after a proxy fence) lets a TMA rewrite the codes
+          mbar_arrive(&empty_W[ws]);
+          // every thread publishes its own row: its stores, the fence that makes them
+          // visible to the tensor core's (async proxy) reads, then its arrival
           fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_A[as]);
+          mbar_arrive(&full_A[as]);
         } else {
           // LoRA weight-side stage: c in [ls*64, ls*64+64), value = src(c mod r) for c < 2r
           const int ls = j - nmain;
@@ -607,8 +632,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_A[as]);
+          mbar_arrive(&full_A[as]);
         }
       }
     }

@@ -199,9 +199,10 @@ size_t qlora_linear_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int
  * device memory of every GPU that loads it (held until the process exits).
  * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - Returns QLORA_ERR_WORKSPACE, before launching anything, when the call
- *     needs more scratch than that (the need grows with M, N*K/16 and r;
- *     4096 tokens on an 11008 x 4096 weight with r = 16 needs about 9 MB; at
- *     r = 16 the first calls that do not fit come at about 36 k tokens).
+ *     needs more scratch than that (the need grows with M and r, plus up to
+ *     9.7 MB for the split partial tiles of the GEMM's last round; 4096 tokens on
+ *     a 4096 x 4096 weight with r = 16 need about 9.6 MB; at r = 16 the first
+ *     calls that do not fit come at about 55 k tokens).
  *   - The first call on each device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture on the device.

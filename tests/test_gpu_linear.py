@@ -298,3 +298,60 @@ def test_capture_before_any_eager_call(q):
     for got, want in zip(outs, ref):
         assert torch.equal(got.view(torch.int16) if got.dtype == torch.bfloat16 else got.view(torch.int32),
                            want.view(torch.int16) if want.dtype == torch.bfloat16 else want.view(torch.int32))
+
+
+@pytest.mark.parametrize("N,K", [(22016, 8192), (4096, 4096)])
+def test_full_output_repeated_against_fp32_gemm(q, N, K):
+    """Every element of Y and dX, over five repeated calls, against an fp32 cuBLAS
+    product (TF32 off) of the same bf16 operands and the library's dequantized weight
+    (whose bits the tests above pin to the oracle).  The oracle checks sample rows at
+    this size; this check covers every tile of every call, so a pipeline race that
+    corrupts one tile now and then cannot hide.  Bound per element: one bf16 ulp of
+    the reference plus the fp32 accumulation floor of helpers.bf16_ulp_check."""
+    import torch
+    tf32 = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        _full_output_check(q, N, K)
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = tf32
+
+
+def _full_output_check(q, N, K):
+    import torch
+    M, r = (8192, 64) if N > 8192 else (4096, 16)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(17)
+    W = (torch.randn(N, K, generator=g, device="cuda") * 0.015).to(torch.bfloat16)
+    X = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
+    dY = torch.randn(M, N, generator=g, device="cuda").to(torch.bfloat16)
+    A = (torch.randn(K, r, generator=g, device="cuda") / r).to(torch.bfloat16)
+    B = (torch.randn(r, N, generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+    s = 0.25
+    Wq = q.nf4_quantize(W)
+    Wd = q.nf4_dequant(Wq).float()
+    del W
+    Xf, Af, Bf, dYf = X.float(), A.float(), B.float(), dY.float()
+    Yref = Xf @ Wd.T + s * ((Xf @ Af) @ Bf)
+    dXref = dYf @ Wd + s * ((dYf @ Bf.T) @ Af.T)
+    del Xf, dYf
+
+    def bound(ref, contraction):
+        mag = ref.abs()
+        ulp = torch.exp2(torch.floor(torch.log2(mag.clamp_min(1e-38))) - 7)
+        rms = float(ref.square().mean().sqrt())
+        return ulp + 4.0 * (contraction ** 0.5) * 2.0 ** -23 * rms
+
+    by, bdx = bound(Yref, K + 2 * r), bound(dXref, N + 2 * r)
+    ws = q.make_workspace(M, N, K, r, X.device)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    XA = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    for call in range(5):
+        q.linear_fwd(X, Wq, A, B, s, workspace=ws, Y=Y, XA=XA)
+        q.linear_bwd(dY, X, XA, Wq, A, B, s, workspace=ws, dX=dX)
+        torch.cuda.synchronize()
+        assert q.device_status() == (0, 0)
+        ey = ((Y.float() - Yref).abs() > by).sum().item()
+        edx = ((dX.float() - dXref).abs() > bdx).sum().item()
+        assert ey == 0 and edx == 0, (call, ey, edx)

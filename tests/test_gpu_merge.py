@@ -5,10 +5,13 @@ after QLoRA") against the fp64 oracle (oracle.linear.merge_weight).
 The oracle rounds the exact value x = base + s (A B)^T once to bf16.  The kernel
 accumulates (A B)^T in fp32 on the tensor cores (r exact products), forms
 fma(s, acc, base) in fp32 and rounds that to bf16.  Its fp32 value is within
-E = (r + 1) 2^-23 |s| (|A| |B|)^T + 2^-23 |x| of x, so its bf16 result can differ
-from the oracle's only where x lies within E of a bf16 rounding boundary, and then
-by one bf16 step.  The test checks exactly that for every element that differs,
-and that such elements stay rare.  With B = 0 the output is the base itself, bit
+E = (r + 1) 2^-23 |s| (|A| |B|)^T + 2^-23 |x| of x, so its bf16 result g can
+differ from the oracle's only where x lies within E of g's rounding interval:
+|x - g| <= E + half a bf16 step at g.  Near a rounding boundary that is one
+step; where base and adapter term cancel it can be several (x is then tiny
+against the terms, whose fp32 error E stays).  The test checks that condition
+for every element that differs, and that such elements stay rare.  With B = 0
+the output is the base itself, bit
 for bit (for an NF4 base: the standalone dequant's output)."""
 import numpy as np
 import pytest
@@ -33,18 +36,33 @@ def _ordered(bits):
     return np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
 
 
+def _from_ordered(o):
+    o = np.asarray(o, np.int64)
+    return np.where(o < 0, 0x8000 | (-o), o).astype(np.uint16)
+
+
+def _rounding_interval(g_bits):
+    """The interval of reals that round (nearest) to each bf16 value: halfway to
+    its neighbours on either side (asymmetric at a power of two)."""
+    o = _ordered(g_bits)
+    v = H.onf4.bf16_to_f32(g_bits).astype(np.float64)
+    lo = H.onf4.bf16_to_f32(_from_ordered(o - 1)).astype(np.float64)
+    hi = H.onf4.bf16_to_f32(_from_ordered(o + 1)).astype(np.float64)
+    return 0.5 * (v + lo), 0.5 * (v + hi)
+
+
 def _check_merge(got, want, Wb, A, B, s, r):
-    steps = np.abs(_ordered(got) - _ordered(want))
-    assert steps.max() <= 1, "more than one bf16 step from the oracle"
-    bad = np.nonzero(steps.ravel())[0]
+    bad = np.nonzero(got.ravel() != want.ravel())[0]
     if bad.size:
         x = (olin.as_f64(Wb) + s * (olin.as_f64(A) @ olin.as_f64(B)).T).ravel()[bad]
         mag = (np.abs(olin.as_f64(A)) @ np.abs(olin.as_f64(B))).T.ravel()[bad]
         E = (r + 1) * 2.0 ** -23 * abs(s) * mag + 2.0 ** -23 * np.abs(x)
-        g = H.onf4.bf16_to_f32(got.ravel()[bad]).astype(np.float64)
-        w = H.onf4.bf16_to_f32(want.ravel()[bad]).astype(np.float64)
-        boundary = 0.5 * (g + w)                       # the rounding boundary between them
-        assert np.all(np.abs(x - boundary) <= E), "a difference not explained by fp32 rounding"
+        lo, hi = _rounding_interval(got.ravel()[bad])
+        dist = np.maximum(0.0, np.maximum(lo - x, x - hi))   # from x to where the GPU value rounds from
+        assert np.all(dist <= E), "a difference not explained by fp32 rounding"
+        steps = np.abs(_ordered(got.ravel()[bad]) - _ordered(want.ravel()[bad]))
+        far = steps > 1                               # only where base and adapter cancel
+        assert np.all(np.abs(x[far]) < 2.0 ** -6 * abs(s) * mag[far] + 1e-30)
     assert bad.size <= max(8, got.size // 2000), (bad.size, got.size)
     return bad.size
 

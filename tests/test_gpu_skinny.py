@@ -100,3 +100,45 @@ def test_few_tokens_beyond_skinny_plan(q):
     p = linear_problem(3, 128, 65536, 8, 16.0, 0.02, seed=5, with_dy=False)
     Yb, XA = _fwd(q, p)
     _check(p, Yb, XA)
+
+
+@pytest.mark.parametrize("M,D,r", [(1, 4096, 16), (4, 2048, 64), (16, 1024, 8)])
+def test_skinny_dependent_chain(q, M, D, r):
+    """Consecutive few-token calls where each call's X is the previous call's Y (square
+    weights, so the shapes chain).  Back-to-back on one stream, and replayed from a CUDA
+    graph, the outputs equal those of calls separated by a device synchronize, bit for
+    bit: a call reads its X only after the previous call's weight pass has finished,
+    although its own weight pass may launch before that."""
+    import torch
+    layers = []
+    for i in range(6):
+        p = linear_problem(M, D, D, r, 2.0 * r, 0.02, seed=100 + i, with_dy=False)
+        layers.append((q.nf4_quantize(H.bits_to_dev(p.W)), H.bits_to_dev(p.A), H.bits_to_dev(p.B), p.s))
+    X0 = H.bits_to_dev(linear_problem(M, D, D, r, 2.0 * r, 0.02, seed=99, with_dy=False).X)
+    ws = q.make_workspace(M, D, D, r, X0.device)
+    outs = [torch.empty(M, D, dtype=torch.bfloat16, device="cuda") for _ in layers]
+
+    def chain(sync):
+        x = X0
+        for (Wq, A, B, s), Y in zip(layers, outs):
+            q.linear_fwd(x, Wq, A, B, s, workspace=ws, Y=Y, want_xa=False)
+            if sync:
+                torch.cuda.synchronize()
+            x = Y
+
+    chain(True)
+    ref = [o.clone() for o in outs]
+    for o in outs:
+        o.zero_()
+    chain(False)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(outs, ref))
+    for o in outs:
+        o.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        chain(False)
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.device_status() == (0, 0)
+    assert all(torch.equal(a, b) for a, b in zip(outs, ref))
