@@ -617,6 +617,7 @@ def main():
         raise RuntimeError(f"device status {code} flags {flags} after timing")
     value = world * wl.flops / (med * 1e-3) / 1e12
     clocks = clk.summary()
+    units = q.gemm_units()
 
     # ---- per-kernel breakdown and the dominant kernel's roofline (second pass)
     kernels, by, launches_per_step = kernel_profile(q, torch, wl.run, args.steps, flush, stream, barrier)
@@ -662,7 +663,8 @@ def main():
                            "lora_alpha": wld["alpha"], "parallelism": f"dp{world}",
                            "l2": "flushed (256 MiB write) before every timed step",
                            "step_time": "median of the timed steps",
-                           "flops_per_step_per_gpu": workload_flops(HEADLINE)},
+                           "flops_per_step_per_gpu": workload_flops(HEADLINE),
+                           "gemm_units": {"ctas": units[0], "pairs": units[1]}},
                 "roofline": roof, "cpu_baseline": cpu_baseline, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "kernels": kernels,
                 "other_workloads": others, "subpaths": subpaths}

@@ -22,6 +22,8 @@ from .api import (  # noqa: F401
     device_status,
     selftest_wait_timeout,
     set_wait_limit_us,
+    set_gemm_pairing,
+    gemm_units,
     profile_enable,
     profile_read,
 )
@@ -29,5 +31,5 @@ from .api import (  # noqa: F401
 __all__ = [
     "NF4Weight", "nf4_levels", "nf4_bytes", "nf4_empty", "nf4_empty_single", "nf4_quantize", "nf4_dequant", "nf4_merge",
     "workspace_bytes", "make_workspace", "pack_keep_mask", "linear_fwd", "linear_bwd", "device_status",
-    "selftest_wait_timeout", "set_wait_limit_us", "profile_enable", "profile_read",
+    "selftest_wait_timeout", "set_wait_limit_us", "set_gemm_pairing", "gemm_units", "profile_enable", "profile_read",
 ]

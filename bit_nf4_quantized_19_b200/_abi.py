@@ -73,6 +73,8 @@ SIGNATURES = {
     "qlora_get_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "qlora_selftest_wait_timeout": (_int, [_u32, _vp]),
     "qlora_set_wait_limit_us": (_u32, [_u32]),
+    "qlora_set_gemm_pairing": (_int, [_int]),
+    "qlora_gemm_units": (_int, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "qlora_profile_enable": (_int, [_int]),
     "qlora_profile_read": (_int, [_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float)]),
 }

@@ -252,6 +252,18 @@ def set_wait_limit_us(limit_us: int) -> int:
     return int(_abi.lib().qlora_set_wait_limit_us(limit_us))
 
 
+def gemm_units() -> tuple:
+    """(single CTAs, CTA pairs) the fused GEMM runs on this device."""
+    a, b = ctypes.c_int(0), ctypes.c_int(0)
+    _abi.check(_abi.lib().qlora_gemm_units(ctypes.byref(a), ctypes.byref(b)), "qlora_gemm_units")
+    return a.value, b.value
+
+
+def set_gemm_pairing(enable: bool) -> bool:
+    """Two-CTA (256-row) GEMM tiles where the output width allows; returns the previous setting."""
+    return bool(_abi.lib().qlora_set_gemm_pairing(1 if enable else 0))
+
+
 def profile_enable(on: bool = True) -> None:
     """Record CUDA events around every launch of the library's kernels."""
     _abi.check(_abi.lib().qlora_profile_enable(1 if on else 0), "qlora_profile_enable")

@@ -78,6 +78,21 @@ QDEV bool wait_bar(uint64_t *bar, uint32_t parity, const Waiter &w) {
   }
 }
 
+// ------------------------------------------------------------------ global flags
+QDEV uint32_t ld_acquire_u32(const unsigned int *a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+QDEV void red_release_add_u32(unsigned int *a, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+QDEV uint32_t atom_acq_rel_add_u32(unsigned int *a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+  return old;
+}
+
 // ------------------------------------------------------------------ clusters
 QDEV uint32_t cluster_ctarank() {
   uint32_t r;
@@ -92,6 +107,16 @@ QDEV uint32_t map_rank(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
+}
+// Arrive on the barrier at the same offset in CTA `rank` of the cluster (default
+// semantics, as a local arrival has).  A cluster-scope release on this arrival costs
+// about 1200 cycles on B200, more than one pipeline stage of the fused GEMM; what an
+// arrival hands over was ordered by its own producers (shared-memory writes fenced to
+// the async proxy, or TMEM reads completed and fenced) before the arriving thread
+// observed their barrier phases.
+QDEV void mbar_arrive_remote(uint64_t *local_bar, uint32_t rank) {
+  const uint32_t a = map_rank(smem_u32(local_bar), rank);
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
 }
 QDEV float ld_dsmem_f32(uint32_t addr) {
   float v;
@@ -140,6 +165,38 @@ QDEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 QDEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 QDEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// The CTA-pair forms (cta_group::2): TMEM allocated at the same address in both CTAs
+// of the pair by warp 1 of each; MMAs of M = 256 issued by the pair's leader, which
+// read A rows 128..255 and B rows 128..255 (the N half) from the peer's shared memory
+// at the leader's offsets and write the peer's TMEM; commits that arrive on the barrier
+// at the same offset in every CTA of the mask.
+QDEV void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+QDEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+QDEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+QDEV void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+QDEV void mma_commit_pair(uint64_t *bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulator.
 // No "memory" clobber: the operands are read asynchronously and ordered by the

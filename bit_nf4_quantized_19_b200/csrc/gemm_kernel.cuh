@@ -32,6 +32,19 @@
 //                 then the LoRA weight tiles.
 // Every wait is bounded (see Waiter); a wait that runs out aborts the block.
 //
+// CTA pairs (cta_group::2, clusters of two; output widths that are multiples of 256):
+// a tile is 256 weight rows x 256 tokens.  Each CTA dequantizes its own 128 weight
+// rows and loads its own 128 tokens of the activation tile, both into its own shared
+// memory at the same offsets; the pair's leader (rank 0) issues one M = 256, N = 256
+// product per K step over both CTAs' operands, writing each CTA's 128 rows into that
+// CTA's TMEM, and its commits arrive on the barrier at the same offset in both CTAs.
+// The peer's warp 1 passes each stage's readiness (its own 128 dequant arrivals and
+// its own activation copy) on to the leader's full_B with a remote arrival; the
+// peer's epilogue warps free the accumulator on the leader's tmem_empty.  Per
+// CTA, the tensor core reads half as many activation bytes per weight byte as a
+// single CTA does (the two halves of N are exchanged between the pair), and the
+// activation tile crosses L2 once per 256 weight rows instead of once per 128.
+//
 // Last-wave split: with T tiles on G persistent CTAs, T mod G tiles are left for a
 // last round in which most SMs would idle.  When at most G/2 remain, each of them
 // is split along the contraction into two halves taken by CTAs 2i and 2i+1 (the
@@ -52,30 +65,37 @@ constexpr int kGemmThreads = 512;
 constexpr int kBN = 256;                  // tokens per tile (MMA N)
 constexpr int kWT = 128;                  // weight-side rows per tile (MMA M)
 constexpr int kBK = 64;                   // contraction per stage (one quant block)
-#ifndef QLORA_GEMM_STAGES
-#define QLORA_GEMM_STAGES 4
-#endif
 #ifndef QLORA_GEMM_STAGES_W
 #define QLORA_GEMM_STAGES_W 6
 #endif
-// The MMA stages: one ring of (activation tile, dequantized weight tile) pairs,
-// released by a single commit per stage.
-constexpr int kStagesB = QLORA_GEMM_STAGES;     // activation tiles (32 KB each)
-constexpr int kStagesA = QLORA_GEMM_STAGES;     // dequantized weight tiles (16 KB each)
 constexpr int kStagesW = QLORA_GEMM_STAGES_W;   // packed code + constant ring (4.5 KB stages)
-constexpr int kBStageBytes = kBN * 128;   // 32 KB
-constexpr int kAStageBytes = kWT * 128;   // 16 KB
+constexpr int kAStageBytes = kWT * 128;   // 16 KB: 128 weight rows x 64 values
 constexpr int kWStageBytes = 4096;        // packed codes of one stage
 constexpr int kSStageBytes = 512;         // 128 fp32 block constants of one stage
 constexpr uint32_t kSplitArrive = 1u;     // split-tile counter: one per arriving half
 constexpr uint32_t kSplitReady = 16u;     // added once the first half's partial is stored
 constexpr int kTmemCols = 512;            // two 256-column fp32 accumulators
 
-constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStagesB * kBStageBytes +
-                               kStagesA * kAStageBytes + kStagesW * (kWStageBytes + kSStageBytes) +
-                               1024 /*barriers, flags, levels*/;
+constexpr int kMaxStagesAB = 6;
+
+// The MMA stages: one ring of (activation tile, dequantized weight tile) pairs,
+// released by a single commit per stage.  A CTA pair loads half the token tile per
+// CTA, so its stages are half as large and the ring is deeper.
+template <bool PAIR>
+struct GemmShape {
+  static constexpr int kStagesAB = PAIR ? 6 : 4;
+  static constexpr int kBRows = PAIR ? kBN / 2 : kBN;    // tokens of the activation tile in this CTA
+  static constexpr int kBStageBytes = kBRows * 128;       // 16 or 32 KB
+  static constexpr int kTileRows = PAIR ? 2 * kWT : kWT;  // weight-side rows of one tile
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStagesAB * (kBStageBytes + kAStageBytes) +
+                                    kStagesW * (kWStageBytes + kSStageBytes) + 1024 /*barriers, flags*/;
+};
+constexpr int kGemmSmemBytes = GemmShape<false>::kSmemBytes > GemmShape<true>::kSmemBytes
+                                   ? GemmShape<false>::kSmemBytes
+                                   : GemmShape<true>::kSmemBytes;
 static_assert(kGemmSmemBytes <= 227 * 1024, "GEMM shared memory exceeds the per-CTA limit");
-static_assert(kStagesW <= 32 && kStagesB <= 32, "ring bookkeeping uses 32-bit masks");
+static_assert(GemmShape<true>::kStagesAB <= kMaxStagesAB && GemmShape<false>::kStagesAB <= kMaxStagesAB, "");
+static_assert(kStagesW <= 32 && kMaxStagesAB <= 32, "ring bookkeeping uses 32-bit masks");
 static_assert(kStagesW % 2 == 0, "the two weight producer warps each keep to the slots of one parity");
 
 enum GemmMode : int { kModeFwd = 0, kModeDx = 1 };
@@ -84,7 +104,8 @@ struct GemmParams {
   int M;             // tokens
   int n_out;         // output row length (N for fwd, K for dX)
   int num_m_tiles;   // ceil(M / 256)
-  int num_w_tiles;   // weight-side tiles: N/128 (fwd) or K/128 (dX)
+  int num_w_tiles;   // weight-side tiles: n_out / 128 (single CTA) or n_out / 256 (CTA pair)
+  int group_m;       // token tiles per raster group (see tile_coords)
   int kb_main;       // main stages: K/64 (fwd) or N/64 (dX)
   int kb_lora;       // LoRA stages: ceil(2r / 64)
   int r;
@@ -95,11 +116,11 @@ struct GemmParams {
   const uint16_t *lora_w;  // fwd: B [r, N];  dX: A [K, r]
   uint16_t *out;     // Y [M, N] or dX [M, K]
   uint64_t limit_ns;
-  int split_base;    // first tile of the split last round (a multiple of the grid size)
+  int split_base;    // first tile of the split last round (a multiple of the unit count)
   int split_count;   // tiles split into two contraction halves (0: no split)
   int kb_mid;        // first main stage of the second half
-  float *scratch;    // [split_count][128][256] fp32 partial tile of the half that finishes first
-  unsigned int *flags;   // [split_count] arrival counters, zero at launch
+  float *scratch;    // [split_count][tile rows / 128][128][256] fp32 partials of the half that arrives first
+  unsigned int *flags;   // [split_count][tile rows / 128] arrival counters, zero at launch
   // dX under adapter-input dropout (null otherwise): the keep mask of X [M, K], bit-packed
   // (element m K + k in bit (m K + k) mod 32 of word (m K + k) / 32).  The adapter term
   // then gets its own accumulator and is added as keep * keep_scale * term per element.
@@ -108,16 +129,23 @@ struct GemmParams {
   float levels[16];
 };
 
-// The work items of this CTA: whole tiles blockIdx.x + i*G below split_base, then
-// (when a last round is split) one half of tile split_base + blockIdx.x/2: part 1
-// = main stages [0, kb_mid), part 2 = [kb_mid, kb_main) plus the LoRA stages.
+// The work items of a unit (a CTA, or a CTA pair) u of G: whole tiles u + i*G below
+// split_base, then (when a last round is split) one half of tile split_base + u/2:
+// part 1 = main stages [0, kb_mid), part 2 = [kb_mid, kb_main) plus the LoRA stages.
 struct GemmItem {
   int tile, kb0, kb1, part;
   bool lora;
 };
 
+// The unit this CTA belongs to, and the number of units.
+template <bool PAIR>
+QDEV int gemm_unit() { return PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x); }
+template <bool PAIR>
+QDEV int gemm_units() { return PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x); }
+
+template <bool PAIR>
 QDEV bool gemm_item(const GemmParams &p, int num_tiles, int it, GemmItem &w) {
-  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  const int G = gemm_units<PAIR>(), b = gemm_unit<PAIR>();
   const int whole_end = p.split_count ? p.split_base : num_tiles;
   const int t = b + it * G;
   if (t < whole_end) {
@@ -133,18 +161,20 @@ QDEV bool gemm_item(const GemmParams &p, int num_tiles, int it, GemmItem &w) {
   return true;
 }
 
-QDEV uint32_t ld_acquire_u32(const unsigned int *a) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-QDEV void red_release_add_u32(unsigned int *a, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
-}
-QDEV uint32_t atom_acq_rel_add_u32(unsigned int *a, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
-  return old;
+// Token tile and weight-side tile of tile index t.  Tiles are taken in groups of
+// group_m token tiles: within a group the token tile varies fastest, so the CTAs
+// running at the same time share group_m activation tiles (kept in L2 while the group
+// sweeps the weight) and each weight tile they stream serves group_m of them, instead
+// of one activation tile against every weight tile of the layer (which re-reads the
+// whole weight from DRAM once per token tile when it does not fit in L2).
+QDEV void tile_coords(const GemmParams &p, int t, int &mt, int &wt) {
+  const int per_group = p.group_m * p.num_w_tiles;
+  const int grp = t / per_group;
+  const int m_base = grp * p.group_m;
+  const int gm = min(p.group_m, p.num_m_tiles - m_base);
+  const int idx = t - grp * per_group;
+  mt = m_base + idx % gm;
+  wt = idx / gm;
 }
 
 // One weight producer warp's walk over the W stages it owns (global W stage
@@ -152,7 +182,7 @@ QDEV uint32_t atom_acq_rel_add_u32(unsigned int *a, uint32_t v) {
 // constants kept incrementally: slot idx = lane + 32 i holds
 //   fwd: weight row w0 + idx, block kb;
 //   dX:  weight row kb*64 + (idx & 63), block w0/64 + (idx >> 6).
-template <int MODE>
+template <int MODE, bool PAIR>
 struct WStageCursor {
   bool have;
   int it, kb0, n, j, w0;
@@ -162,11 +192,13 @@ struct WStageCursor {
 
   QDEV void enter(const GemmParams &p, int num_tiles, int lane) {
     GemmItem w;
-    have = gemm_item(p, num_tiles, it, w);
+    have = gemm_item<PAIR>(p, num_tiles, it, w);
     if (!have) return;
     kb0 = w.kb0;
     n = w.kb1 - w.kb0;
-    w0 = (w.tile % p.num_w_tiles) * kWT;
+    int mti, wti;
+    tile_coords(p, w.tile, mti, wti);
+    w0 = wti * GemmShape<PAIR>::kTileRows + (PAIR ? static_cast<int>(cluster_ctarank()) * kWT : 0);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int idx = lane + 32 * i;
@@ -213,24 +245,27 @@ struct WStageCursor {
 
 QDEV void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,   // X or dY, bf16 [M, contraction]
                       const __grid_constant__ CUtensorMap tm_codes, // packed codes, u8 [N, K/2]
                       const __grid_constant__ CUtensorMap tm_lora,  // hi/lo LoRA operand, bf16 [M, 2r]
                       const __grid_constant__ GemmParams p) {
+  using S = GemmShape<PAIR>;
+  constexpr int kStages = S::kStagesAB;
+  constexpr int kBStage = S::kBStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sB = smem;
-  uint8_t *sA = sB + kStagesB * kBStageBytes;
-  uint8_t *sW = sA + kStagesA * kAStageBytes;
+  uint8_t *sA = sB + kStages * kBStage;
+  uint8_t *sW = sA + kStages * kAStageBytes;
   float *sS = reinterpret_cast<float *>(sW + kStagesW * kWStageBytes);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sS + kStagesW * (kSStageBytes / 4));
-  uint64_t *full_B = bars;                  // activation tile landed (TMA)
-  uint64_t *full_A = full_B + kStagesB;     // dequantized tile written (128 thread arrivals)
-  uint64_t *empty_A = full_A + kStagesA;    // MMAs of the stage done: both tiles free
-  uint64_t *full_W = empty_A + kStagesA;
+  uint64_t *full_B = bars;                  // activation tile landed (and, at a pair's leader, the peer's stage)
+  uint64_t *full_A = full_B + kStages;      // dequantized tile written (128 thread arrivals)
+  uint64_t *empty_A = full_A + kStages;     // MMAs of the stage done: both tiles free
+  uint64_t *full_W = empty_A + kStages;
   uint64_t *empty_W = full_W + kStagesW;
   uint64_t *tmem_full = empty_W + kStagesW;
   uint64_t *tmem_empty = tmem_full + 2;
@@ -243,18 +278,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int row_off = static_cast<int>(rank) * kWT;           // this CTA's weight rows in a tile
+  const int tok_off = static_cast<int>(rank) * S::kBRows;     // this CTA's tokens of a tile
 
   if (tid == 0) {
-    // full_A: one arrival per dequant thread, each after its own stores and proxy fence
-    for (int i = 0; i < kStagesA; ++i) {
-      mbar_init(&full_B[i], 1);
+    // full_B: this CTA's expect_tx arrival, plus at a pair's leader the peer's forwarded
+    // "my stage is ready"; full_A: one arrival per dequant thread of this CTA, each after
+    // its own stores and proxy fence
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full_B[i], (PAIR && leader) ? 2 : 1);
       mbar_init(&full_A[i], 128);
       mbar_init(&empty_A[i], 1);
     }
     // full_W: the TMA's expect_tx arrival plus one per lane of the weight producer;
     // empty_W: one per consumer thread, each once it has used what it read
     for (int i = 0; i < kStagesW; ++i) { mbar_init(&full_W[i], 33); mbar_init(&empty_W[i], 128); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 4); }
+    // tmem_empty: one per epilogue warp (both CTAs' at a pair's leader)
+    for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], PAIR ? 8 : 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -266,11 +308,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tmap(&tm_lora);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // a pair's barriers are initialized before either CTA arrives on the other's
+  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const Waiter wt{abort_flag, p.limit_ns};
@@ -285,25 +334,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t armedB = 0, lastB = 0;          // bit s: armed at least once / parity of last arming
       bool ok = true;
       GemmItem w;
-      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
-        const int m0 = (w.tile / p.num_w_tiles) * kBN;
+      for (int it = 0; ok && gemm_item<PAIR>(p, num_tiles, it, w); ++it) {
+        int mti, wti;
+        tile_coords(p, w.tile, mti, wti);
+        const int m0 = mti * kBN + tok_off;
         const int nmain = w.kb1 - w.kb0, nst = nmain + (w.lora ? p.kb_lora : 0);
         for (int j = 0; j < nst; ++j) {
           if (!wait_bar(&empty_A[bs], bph ^ 1u, wt)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_B[bs], kBStageBytes);
+          mbar_arrive_expect_tx(&full_B[bs], kBStage);
           if (j < nmain)
-            tma_load_2d(sB + bs * kBStageBytes, &tm_act, &full_B[bs], (w.kb0 + j) * kBK, m0);
+            tma_load_2d(sB + bs * kBStage, &tm_act, &full_B[bs], (w.kb0 + j) * kBK, m0);
           else
-            tma_load_2d(sB + bs * kBStageBytes, &tm_lora, &full_B[bs], (j - nmain) * kBK, m0);
+            tma_load_2d(sB + bs * kBStage, &tm_lora, &full_B[bs], (j - nmain) * kBK, m0);
           armedB |= 1u << bs;
           lastB = (lastB & ~(1u << bs)) | (bph << bs);
-          if (++bs == kStagesB) { bs = 0; bph ^= 1u; }
+          if (++bs == kStages) { bs = 0; bph ^= 1u; }
         }
       }
-      // Every issued copy lands before the block may exit (bounded).
+      // Every issued copy lands before the block may exit (bounded).  At a pair's
+      // leader a phase also needs the peer's forwarded arrival, which comes once the
+      // peer's own copy of that stage has landed, or not at all after an abort: the
+      // wait is bounded either way, and this CTA's copies have landed when it ends.
       volatile int no_abort = 0;
       const Waiter final_wt{&no_abort, p.limit_ns};
-      for (int s = 0; s < kStagesB; ++s)
+      for (int s = 0; s < kStages; ++s)
         if (armedB & (1u << s)) wait_bar(&full_B[s], (lastB >> s) & 1u, final_wt);
     }
   } else if (warp == 2 || warp == 3) {
@@ -314,14 +368,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the raw constants of a warp's next stage are requested before it waits for the
     // current one.
     const uint32_t wp = static_cast<uint32_t>(warp - 2);
-    WStageCursor<MODE> cur;
+    WStageCursor<MODE, PAIR> cur;
     cur.start(p, num_tiles, lane, wp);
     uint32_t qc[4] = {0u, 0u, 0u, 0u}, qn[4] = {0u, 0u, 0u, 0u};
     float sc[4] = {0.f, 0.f, 0.f, 0.f}, sn[4] = {0.f, 0.f, 0.f, 0.f};
     if (cur.have) cur.load(p, qc, sc);
     uint32_t armedW = 0, lastW = 0;
     while (cur.have) {
-      WStageCursor<MODE> nx = cur;
+      WStageCursor<MODE, PAIR> nx = cur;
       nx.advance(p, num_tiles, lane);
       if (nx.have) nx.load(p, qn, sn);
       const uint32_t c = cur.c0 + static_cast<uint32_t>(cur.j);
@@ -359,15 +413,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int s = 0; s < kStagesW; ++s)
         if (armedW & (1u << s)) wait_bar(&full_W[s], (lastW >> s) & 1u, final_wt);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 && leader) {
     // ------------------------------------------------------------ MMA issuer
     // A lean loop: descriptors of stage 0 are built once; a stage adds its byte
     // offset >> 4 to the start-address field, a K=16 step adds 32 B (K-major)
     // or 4096 B (MN-major, two 8-row groups) >> 4; one commit per stage frees
-    // both tiles of the stage.
+    // both tiles of the stage (in both CTAs of a pair).
     if (lane == 0) {
-      constexpr uint32_t idesc_main = make_idesc_bf16(kWT, kBN, MODE == kModeDx, false);
-      constexpr uint32_t idesc_lora = make_idesc_bf16(kWT, kBN, MODE == kModeFwd, false);
+      constexpr int kM = PAIR ? 2 * kWT : kWT;
+      constexpr uint32_t idesc_main = make_idesc_bf16(kM, kBN, MODE == kModeDx, false);
+      constexpr uint32_t idesc_lora = make_idesc_bf16(kM, kBN, MODE == kModeFwd, false);
       constexpr uint32_t a_step_main = (MODE == kModeDx) ? (4096u >> 4) : (32u >> 4);
       constexpr uint32_t a_step_lora = (MODE == kModeFwd) ? (4096u >> 4) : (32u >> 4);
       const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
@@ -380,11 +435,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // adapter term in [256, 512)
       const bool two_acc = (MODE == kModeDx) && (p.keep32 != nullptr);
       const int nacc = two_acc ? 1 : 2;
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t accumulate) {
+        if constexpr (PAIR) mma_bf16_ss_pair(d, ad, bd, idesc, accumulate);
+        else mma_bf16_ss(d, ad, bd, idesc, accumulate);
+      };
+      auto commit = [&](uint64_t *bar) {
+        if constexpr (PAIR) mma_commit_pair(bar, static_cast<uint16_t>(0x3));
+        else mma_commit(bar);
+      };
       int st = 0, acc = 0;
       uint32_t ph = 0, accph = 0;
       bool ok = true;
       GemmItem w;
-      for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
+      for (int it = 0; ok && gemm_item<PAIR>(p, num_tiles, it, w); ++it) {
         if (!wait_bar(&tmem_empty[acc], accph ^ 1u, wt)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
@@ -393,31 +456,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = ad_main0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
-          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStageBytes >> 4));
+          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStage >> 4));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(d_tmem, ad + k * a_step_main, bd + k * 2, idesc_main, (kb | k) ? 1u : 0u);
-          mma_commit(&empty_A[st]);
-          if (++st == kStagesA) { st = 0; ph ^= 1u; }
+            mma(d_tmem, ad + k * a_step_main, bd + k * 2, idesc_main, (kb | k) ? 1u : 0u);
+          commit(&empty_A[st]);
+          if (++st == kStages) { st = 0; ph ^= 1u; }
         }
         for (int ls = 0; ok && w.lora && ls < kb_lora; ++ls) {
           if (!wait_bar(&full_A[st], ph, wt) || !wait_bar(&full_B[st], ph, wt)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = ad_lora0 + static_cast<uint64_t>(st * (kAStageBytes >> 4));
-          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStageBytes >> 4));
+          const uint64_t bd = bd0 + static_cast<uint64_t>(st * (kBStage >> 4));
           const int nk = min(4, lora_steps_total - ls * 4);
           for (int k = 0; k < nk; ++k)
-            mma_bf16_ss(d_lora, ad + k * a_step_lora, bd + k * 2, idesc_lora,
-                        (two_acc && (ls | k) == 0) ? 0u : 1u);
-          mma_commit(&empty_A[st]);
-          if (++st == kStagesA) { st = 0; ph ^= 1u; }
+            mma(d_lora, ad + k * a_step_lora, bd + k * 2, idesc_lora, (two_acc && (ls | k) == 0) ? 0u : 1u);
+          commit(&empty_A[st]);
+          if (++st == kStages) { st = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(&tmem_full[acc]);
+        commit(&tmem_full[acc]);
         if (++acc == nacc) { acc = 0; accph ^= 1u; }
       }
-      // All issued MMAs complete before TMEM is released (bounded).
-      mma_commit(drain);
+      // All issued MMAs complete before TMEM (and, in a pair, the peer's operands) is
+      // released (bounded).
+      commit(drain);
+      volatile int no_abort = 0;
+      const Waiter final_wt{&no_abort, p.limit_ns};
+      wait_bar(drain, 0, final_wt);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair peer: forwarder
+    // The peer's own stage (its dequantized tile, 128 thread arrivals, and its
+    // activation copy) completes on its own barriers; once both have, the stage is
+    // passed on to the leader's full_B of that stage, in stage order.  The peer's
+    // stores were made visible to the tensor core by each thread's proxy fence, and
+    // its copy had landed, before this thread observed the two phases.
+    if (PAIR && lane == 0) {
+      int bs = 0;
+      uint32_t bph = 0;
+      bool ok = true;
+      GemmItem w;
+      for (int it = 0; ok && gemm_item<PAIR>(p, num_tiles, it, w); ++it) {
+        const int nst = (w.kb1 - w.kb0) + (w.lora ? p.kb_lora : 0);
+        for (int j = 0; j < nst; ++j) {
+          if (!wait_bar(&full_A[bs], bph, wt) || !wait_bar(&full_B[bs], bph, wt)) { ok = false; break; }
+          mbar_arrive_remote(&full_B[bs], 0u);
+          if (++bs == kStages) { bs = 0; bph ^= 1u; }
+        }
+      }
+      // the leader's MMAs read this CTA's shared memory and write its TMEM: they
+      // complete before either is released (bounded)
       volatile int no_abort = 0;
       const Waiter final_wt{&no_abort, p.limit_ns};
       wait_bar(drain, 0, final_wt);
@@ -425,21 +514,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant of this warp
-    const int row = q * 32 + lane;      // weight-side row within the tile
+    const int row = q * 32 + lane;      // weight-side row within this CTA's 128
+    constexpr int kParts = S::kTileRows / kWT;                       // 128-row parts per tile
     const bool two_acc = (MODE == kModeDx) && (p.keep32 != nullptr);
     const int nacc = two_acc ? 1 : 2;
     const int64_t keep_words = static_cast<int64_t>(p.n_out) >> 5;   // mask words per token
     int acc = 0;
     uint32_t accph = 0;
     GemmItem w;
-    for (int it = 0; gemm_item(p, num_tiles, it, w); ++it) {
-      const int m0 = (w.tile / p.num_w_tiles) * kBN;
-      const int w0 = (w.tile % p.num_w_tiles) * kWT;
+    for (int it = 0; gemm_item<PAIR>(p, num_tiles, it, w); ++it) {
+      int mti, wti;
+      tile_coords(p, w.tile, mti, wti);
+      const int m0 = mti * kBN;
+      const int w0 = wti * S::kTileRows + row_off;
       // warp-uniform decision: the TMEM loads below are .sync.aligned
       const bool got = __all_sync(0xffffffffu, wait_bar(&tmem_full[acc], accph, wt) ? 1 : 0);
       if (!got) break;
       tc_fence_after();
-      const int sidx = w.tile - p.split_base;                  // split tiles only
+      const int sidx = (w.tile - p.split_base) * kParts + static_cast<int>(rank);   // split tiles only
       float *prow = (w.part != 0) ? p.scratch + (static_cast<int64_t>(sidx) * kWT + row) * kBN : nullptr;
       // role: 0 a whole tile; 1 the first half of a split tile to finish (stores its
       // partial); 2 the second (adds the partial and writes the output)
@@ -531,7 +623,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+      if (lane == 0) {
+        if (PAIR && !leader) mbar_arrive_remote(&tmem_empty[acc], 0u);
+        else mbar_arrive(&tmem_empty[acc]);
+      }
       if (++acc == nacc) { acc = 0; accph ^= 1u; }
     }
   } else if (warp >= 8) {
@@ -544,25 +639,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t a_cnt = 0, w_cnt = 0;      // stages seen so far (all / main only)
     bool ok = true;
     GemmItem w;
-    for (int it = 0; ok && gemm_item(p, num_tiles, it, w); ++it) {
-      const int w0 = (w.tile % p.num_w_tiles) * kWT;
+    for (int it = 0; ok && gemm_item<PAIR>(p, num_tiles, it, w); ++it) {
+      int mti, wti;
+      tile_coords(p, w.tile, mti, wti);
+      const int w0 = wti * S::kTileRows + row_off;
       const int nmain = w.kb1 - w.kb0, nst = nmain + (w.lora ? p.kb_lora : 0);
       for (int j = 0; j < nst; ++j, ++a_cnt) {
         const bool main = j < nmain;
         const uint32_t my_w = w_cnt;
         if (main) ++w_cnt;
         if ((a_cnt & 1u) != static_cast<uint32_t>(grp)) continue;
-        const int as = static_cast<int>(a_cnt % kStagesA);
-        const uint32_t aph = (a_cnt / kStagesA) & 1u;
+        const int as = static_cast<int>(a_cnt % kStages);
+        const uint32_t aph = (a_cnt / kStages) & 1u;
         if (main) {
           const int ws = static_cast<int>(my_w % kStagesW);
           const uint32_t wph = (my_w / kStagesW) & 1u;
           // warp-uniform: the per-warp arrivals below need every lane on the same path.
-          // The A slot first: once it is free the MMA has consumed A stage a_cnt - 4,
-          // so the dequant of W stage my_w - 6 (an earlier stage, whichever warpgroup
-          // took it) has passed its own wait on this W slot, whose barrier is then at
-          // least in the phase this wait names.  (Waiting on full_W first could see a
-          // phase two behind and take the previous parity's completion for this one.)
+          // The A slot first: once it is free the MMA has consumed A stage
+          // a_cnt - kStages and every stage before it, so the dequant of W stage
+          // my_w - kStagesW (an earlier A stage, whichever warpgroup took it) has passed
+          // its own wait on this W slot, whose barrier is then at least in the phase this
+          // wait names.  (Waiting on full_W first could see a phase two behind and take
+          // the previous parity's completion for this one.)
           const bool w_ok = wait_bar(&empty_A[as], aph ^ 1u, wt) && wait_bar(&full_W[ws], wph, wt);
           if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
           uint32_t src, dst;
@@ -640,10 +738,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still arrive on its barriers
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

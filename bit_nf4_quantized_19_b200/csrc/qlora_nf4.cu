@@ -20,16 +20,17 @@ using namespace qlora;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+#ifndef QLORA_GEMM_RASTER_MB
+#define QLORA_GEMM_RASTER_MB 40
+#endif
 constexpr int64_t kSkinnyMaxTokens = 16;   // forward with at most this many tokens: one-launch kernel
 std::atomic<uint32_t> g_wait_limit_us{2000000u};
+std::atomic<int> g_gemm_pairing{1};        // CTA-pair GEMM where the output width allows it
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
-#ifndef QLORA_SKINNY_CLUSTER
-#define QLORA_SKINNY_CLUSTER 8
-#endif
 constexpr int kSkSmemLimit = 200 * 1024;
 
 template <int C>
@@ -41,10 +42,18 @@ cudaError_t set_skinny_attrs() {
   return e;
 }
 
+// Persistent units of the fused GEMM: single CTAs, and CTA pairs (clusters of two)
+// that the device can hold at once with one CTA per SM (0: no pairs).
+struct GemmUnits {
+  int ctas = 148;
+  int pairs = 74;
+};
+
 struct DeviceInfo {
   int sms = 0;
   int major = 0;
   bool gemm_attr_set = false;
+  GemmUnits units;
 };
 
 constexpr int kMaxDevices = 64;
@@ -67,9 +76,13 @@ qlora_status device_info(DeviceInfo **out) {
   }
   if (d.major != 10) return QLORA_ERR_NO_DEVICE;
   if (!d.gemm_attr_set) {
-    if (cudaFuncSetAttribute(qlora_gemm_kernel<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qlora_gemm_kernel<kModeFwd, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGemmSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(qlora_gemm_kernel<kModeFwd, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGemmSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
     if (cudaFuncSetAttribute(lora_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
@@ -87,6 +100,26 @@ qlora_status device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(nf4_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              merge_smem_bytes(2)) != cudaSuccess)
       return QLORA_ERR_CUDA;
+    d.units.ctas = d.sms;
+    d.units.pairs = 0;
+    {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(static_cast<unsigned>(d.sms / 2 * 2), 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = kGemmSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (d.sms >= 2 &&
+          cudaOccupancyMaxActiveClusters(&n, qlora_gemm_kernel<kModeFwd, true>, &cfg) == cudaSuccess && n > 0)
+        d.units.pairs = n < d.sms / 2 ? n : d.sms / 2;
+      (void)cudaGetLastError();
+    }
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -275,17 +308,24 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
 int nn_proj(int r) { return (r + 15) / 16 * 16; }
 int64_t pad8(int64_t m) { return (m + 7) / 8 * 8; }
 
-// Last-wave split of one fused GEMM launch (see gemm_kernel.cuh): the tiles left for
-// the last round are split along the contraction when at most half the grid remains.
+// Shape of one fused GEMM launch (see gemm_kernel.cuh): single CTAs with 128-row weight
+// tiles, or CTA pairs with 256-row tiles when the output width is a multiple of 256;
+// and its last-wave split, where the tiles left for the last round are split along the
+// contraction when at most half the units (CTAs or pairs) remain.
 struct GemmSplit {
+  bool pair = false;
   int base = 0, count = 0;
-  size_t scratch_bytes() const { return static_cast<size_t>(count) * kWT * kBN * 4; }
-  size_t flag_bytes() const { return static_cast<size_t>(count) * 4; }
+  int parts() const { return pair ? 2 : 1; }     // 128-row partial tiles per split tile
+  size_t scratch_bytes() const { return static_cast<size_t>(count) * parts() * kWT * kBN * 4; }
+  size_t flag_bytes() const { return static_cast<size_t>(count) * parts() * 4; }
 };
-GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, int sms) {
+bool gemm_pairable(int64_t n_out, const GemmUnits &u) { return n_out % (2 * kWT) == 0 && u.pairs > 0; }
+GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, const GemmUnits &u, bool pair) {
   GemmSplit g;
-  const int64_t tiles = ((M + kBN - 1) / kBN) * (n_out / kWT);
-  const int64_t grid = tiles < sms ? tiles : sms;
+  g.pair = pair;
+  const int64_t units = pair ? u.pairs : u.ctas;
+  const int64_t tiles = ((M + kBN - 1) / kBN) * (n_out / (pair ? 2 * kWT : kWT));
+  const int64_t grid = tiles < units ? tiles : units;
   if (grid <= 0 || contraction / kBK < 2) return g;
   const int64_t rem = tiles % grid;
   if (rem > 0 && 2 * rem <= grid) {
@@ -294,7 +334,20 @@ GemmSplit gemm_split(int64_t M, int64_t n_out, int64_t contraction, int sms) {
   }
   return g;
 }
+// The variant a call uses, fixed once per call.
+GemmSplit gemm_plan(int64_t M, int64_t n_out, int64_t contraction, const GemmUnits &u) {
+  return gemm_split(M, n_out, contraction, u, g_gemm_pairing.load() != 0 && gemm_pairable(n_out, u));
+}
 size_t split_workspace(const GemmSplit &g) { return align256(g.scratch_bytes()) + align256(g.flag_bytes()); }
+// Workspace sizes do not depend on the variant switch: the larger of the two.
+size_t split_workspace_any(int64_t M, int64_t n_out, int64_t contraction, const GemmUnits &u) {
+  size_t a = split_workspace(gemm_split(M, n_out, contraction, u, false));
+  if (gemm_pairable(n_out, u)) {
+    const size_t b = split_workspace(gemm_split(M, n_out, contraction, u, true));
+    if (b > a) a = b;
+  }
+  return a;
+}
 
 // Scratch of one split GEMM launch, carved from the workspace before the call's first
 // launch: its arrival counters are cleared by the rank-r projection that precedes the
@@ -305,16 +358,16 @@ struct SplitScratch {
   unsigned int *flags = nullptr;
 };
 
-size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
+size_t fwd_workspace(int64_t M, int64_t N, int64_t K, int r, const GemmUnits &u) {
   size_t b = 0;
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T
   b += align256(static_cast<size_t>(M) * 2 * r * 2);           // s*XA hi/lo
   b += align256(static_cast<size_t>(M) * r * 4);               // XA when XA_out is NULL
-  b += split_workspace(gemm_split(M, N, K, sms));              // last-wave partial tiles
+  b += split_workspace_any(M, N, K, u);                      // last-wave partial tiles
   return b + 256;
 }
 
-size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
+size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, const GemmUnits &u) {
   size_t b = 0;
   b += align256(static_cast<size_t>(r) * K * 2);               // A^T (XA recompute)
   b += align256(static_cast<size_t>(M) * r * 4);               // G
@@ -322,7 +375,7 @@ size_t bwd_workspace(int64_t M, int64_t N, int64_t K, int r, int sms) {
   b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*G hi/lo transposed
   b += align256(static_cast<size_t>(2 * r) * pad8(M) * 2);     // s*XA hi/lo transposed
   b += align256(static_cast<size_t>(M) * r * 4);               // XA recomputed
-  b += split_workspace(gemm_split(M, K, N, sms));              // last-wave partial tiles (dX)
+  b += split_workspace_any(M, K, N, u);                      // last-wave partial tiles (dX)
   return b + 256;
 }
 
@@ -436,7 +489,7 @@ qlora_status launch_projection(const uint16_t *act, int64_t M, int64_t C, const 
   p.out_scale = p.out_scale1 = out_scale;
   if (clear && clear->g.count) {
     p.zero = clear->flags;
-    p.zero_n = clear->g.count;
+    p.zero_n = clear->g.count * clear->g.parts();
   }
   p.grad = 0;
   p.r = r;
@@ -493,39 +546,80 @@ qlora_status launch_transpose(const uint16_t *A, int64_t K, int r, uint16_t *AT,
   return cuda_status(cudaGetLastError());
 }
 
-// Few-token forward: one cluster launch, no workspace.  Clusters of C CTAs
-// (power of two, 8 preferred, 16 when the slice would not fit) split K into C
-// slices of ks (a multiple of 256) values.  False when no plan fits: the caller
-// then takes the general path.
-bool skinny_choose(int64_t M, int64_t K, int r, SkinnyPlan &pl) {
-  const int64_t macro = (K + kSkMacro - 1) / kSkMacro;
-  int C = QLORA_SKINNY_CLUSTER;
-  while (C > 1 && C > macro) C >>= 1;
-  for (; C <= kSkMaxCluster; C <<= 1)
-    if (skinny_plan_for(static_cast<int>(M), static_cast<int>(K), r, C, kSkSmemLimit, pl)) return true;
-  return false;
-}
-
-// 16-CTA clusters are not portable: take one only where the device can place it.
-bool skinny_launchable(const SkinnyPlan &pl, int64_t N) {
-  if (pl.C <= 8) return true;
+// Few-token forward: one cluster launch, no workspace.  Clusters of C CTAs split K
+// into C slices of ks (a multiple of 256) values, one cluster per 128 weight rows.
+// C is chosen for the fewest waves of clusters (the device holds only so many at
+// once: the count comes from the occupancy query, cached per plan), then in the order
+// 8, 4, 16, 2, 1.  8 splits give each weight tile the most SMs; fewer splits keep a
+// tall weight (many row tiles) in one wave, where 8 would leave a partial second wave
+// of short-lived CTAs.  False when no plan fits: the caller then takes the general path.
+template <int C>
+cudaError_t skinny_occupancy(int smem, int *n) {
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(pl.C), static_cast<unsigned>(N / kSkRows), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(C), 1, 1);
   cfg.blockDim = dim3(kSkThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(pl.C);
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, qlora_skinny_kernel<16>, &cfg) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
+  return cudaOccupancyMaxActiveClusters(n, qlora_skinny_kernel<C>, &cfg);
+}
+
+std::mutex g_sk_occ_mu;
+std::map<std::pair<int, int>, int> g_sk_occ[kMaxDevices];
+
+// Clusters of plan pl the current device holds at once (0: none).
+int skinny_resident(const SkinnyPlan &pl) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  const std::pair<int, int> key{pl.C, pl.smem};
+  {
+    std::lock_guard<std::mutex> lk(g_sk_occ_mu);
+    auto it = g_sk_occ[dev].find(key);
+    if (it != g_sk_occ[dev].end()) return it->second;
   }
-  return n > 0;
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (pl.C) {
+    case 1: e = skinny_occupancy<1>(pl.smem, &n); break;
+    case 2: e = skinny_occupancy<2>(pl.smem, &n); break;
+    case 4: e = skinny_occupancy<4>(pl.smem, &n); break;
+    case 8: e = skinny_occupancy<8>(pl.smem, &n); break;
+    case 16: e = skinny_occupancy<16>(pl.smem, &n); break;
+    default: break;
+  }
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(g_sk_occ_mu);
+  g_sk_occ[dev][key] = n;
+  return n;
+}
+
+bool skinny_choose(int64_t M, int64_t N, int64_t K, int r, SkinnyPlan &pl) {
+  const int64_t macro = (K + kSkMacro - 1) / kSkMacro;
+  const int64_t row_tiles = N / kSkRows;
+  int64_t best_waves = 0;
+  bool found = false;
+  for (const int C : {8, 4, 16, 2, 1}) {
+    if (C > 1 && C > macro) continue;   // a slice holds at least one 256-value macro-block
+    SkinnyPlan cand{};
+    if (!skinny_plan_for(static_cast<int>(M), static_cast<int>(K), r, C, kSkSmemLimit, cand)) continue;
+    const int resident = skinny_resident(cand);
+    if (resident <= 0) continue;
+    const int64_t waves = (row_tiles + resident - 1) / resident;
+    if (!found || waves < best_waves) {
+      pl = cand;
+      best_waves = waves;
+      found = true;
+    }
+  }
+  return found;
 }
 
 // xa_src is the adapter input (X, or X (.) keep under dropout) and xa_scale the factor of
@@ -624,13 +718,18 @@ qlora_status launch_skinny(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq, 
 template <int MODE>
 qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
                          const uint16_t *lora_act_hl, const uint16_t *lora_w, int r,
-                         uint16_t *out, const SplitScratch &sp, int sms, cudaStream_t st,
+                         uint16_t *out, const SplitScratch &sp, const GemmUnits &u, cudaStream_t st,
                          const uint8_t *keep = nullptr, float keep_scale = 1.0f) {
   const int64_t N = Wq->rows, K = Wq->cols;
+  const int64_t n_out = (MODE == kModeFwd) ? N : K;
   const int64_t contraction = (MODE == kModeFwd) ? K : N;
+  const bool pair = sp.g.pair;
+  if (pair && !gemm_pairable(n_out, u)) return QLORA_ERR_WORKSPACE;
+  // a pair's CTAs each load half of the 256-token activation tile
+  const int b_rows = pair ? kBN / 2 : kBN;
   CUtensorMap tm_act, tm_codes, tm_lora;
   if (!make_map_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, contraction, M, contraction * 2,
-                   kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+                   kBK, b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
   if (MODE == kModeFwd) {
     if (!make_map_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, 32, kWT,
@@ -642,14 +741,22 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
       return QLORA_ERR_CUDA;
   }
   if (!make_map_2d(&tm_lora, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_act_hl, 2 * r, M, 4 * r, kBK,
-                   kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+                   b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
 
   GemmParams p{};
   p.M = static_cast<int>(M);
-  p.n_out = static_cast<int>((MODE == kModeFwd) ? N : K);
+  p.n_out = static_cast<int>(n_out);
   p.num_m_tiles = static_cast<int>((M + kBN - 1) / kBN);
-  p.num_w_tiles = static_cast<int>(((MODE == kModeFwd) ? N : K) / kWT);
+  p.num_w_tiles = static_cast<int>(n_out / (pair ? 2 * kWT : kWT));
+  {
+    // token tiles per raster group: as many activation tiles as fit a share of L2
+    const int64_t act_tile = static_cast<int64_t>(kBN) * contraction * 2;
+    int64_t g = static_cast<int64_t>(QLORA_GEMM_RASTER_MB) * (1 << 20) / act_tile;
+    if (g < 1) g = 1;
+    if (g > p.num_m_tiles) g = p.num_m_tiles;
+    p.group_m = static_cast<int>(g);
+  }
   p.kb_main = static_cast<int>(contraction / kBK);
   p.kb_lora = (2 * r + kBK - 1) / kBK;
   p.r = r;
@@ -663,8 +770,9 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
   const Nf4Tables &T = nf4_tables();
   std::memcpy(p.levels, T.levels, sizeof(p.levels));
   const int tiles = p.num_m_tiles * p.num_w_tiles;
-  const int grid = tiles < sms ? tiles : sms;
-  const GemmSplit g = gemm_split(M, (MODE == kModeFwd) ? N : K, contraction, sms);
+  const int units = pair ? u.pairs : u.ctas;
+  const int grid_units = tiles < units ? tiles : units;
+  const GemmSplit g = gemm_split(M, n_out, contraction, u, pair);
   if (g.count != sp.g.count || g.base != sp.g.base) return QLORA_ERR_WORKSPACE;
   p.split_base = g.base;
   p.split_count = g.count;
@@ -674,8 +782,23 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
   p.keep32 = (MODE == kModeDx) ? reinterpret_cast<const uint32_t *>(keep) : nullptr;
   p.keep_scale = keep_scale;
   LaunchTimer lt(MODE == kModeFwd ? QLORA_K_GEMM_FWD : QLORA_K_GEMM_DX, st);
-  qlora_gemm_kernel<MODE><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_lora, p);
-  return cuda_status(cudaGetLastError());
+  if (!pair) {
+    qlora_gemm_kernel<MODE, false><<<grid_units, kGemmThreads, kGemmSmemBytes, st>>>(tm_act, tm_codes, tm_lora, p);
+    return cuda_status(cudaGetLastError());
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * grid_units), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<MODE, true>, tm_act, tm_codes, tm_lora, p));
 }
 
 // ------------------------------------------------------------------ the linear layer
@@ -706,7 +829,7 @@ qlora_status linear_fwd_impl(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq
   DeviceInfo *d = nullptr;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t N = Wq->rows, K = Wq->cols;
-  const size_t need = fwd_workspace(M, N, K, r, d->sms) + (keep ? mask_workspace(M, K) : 0);
+  const size_t need = fwd_workspace(M, N, K, r, d->units) + (keep ? mask_workspace(M, K) : 0);
   if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   // the adapter input: X, or X (.) keep under dropout (its products then carry 1/(1-p))
@@ -720,23 +843,24 @@ qlora_status linear_fwd_impl(const uint16_t *X, int64_t M, const qlora_nf4_t *Wq
   }
   if (M <= kSkinnyMaxTokens) {
     SkinnyPlan pl{};
-    if (skinny_choose(M, K, r, pl) && skinny_launchable(pl, N)) {
+    if (skinny_choose(M, N, K, r, pl)) {
       float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
       if (!xa) return QLORA_ERR_WORKSPACE;
       return launch_skinny(X, M, Wq, A, B, r, s, Y, xa, pl, stream, xin, xscale);
     }
   }
+
   uint16_t *AT = static_cast<uint16_t *>(ws.take(static_cast<size_t>(r) * K * 2));
   uint16_t *hl = static_cast<uint16_t *>(ws.take(static_cast<size_t>(M) * 2 * r * 2));
   float *xa = XA_out ? XA_out : static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   SplitScratch sp;
-  if (!AT || !hl || !xa || !take_split(ws, gemm_split(M, N, K, d->sms), sp)) return QLORA_ERR_WORKSPACE;
+  if (!AT || !hl || !xa || !take_split(ws, gemm_plan(M, N, K, d->units), sp)) return QLORA_ERR_WORKSPACE;
   // XA = X A (fp32) and s*XA as bf16 hi|lo, the activation side of the LoRA K-steps;
   // the projection also clears the GEMM's split counters
   if ((st = launch_transpose(A, K, r, AT, d->sms, stream)) != QLORA_OK) return st;
   if ((st = launch_projection(xin, M, K, AT, r, s, xa, hl, nullptr, d->sms, stream, &sp, xscale)) != QLORA_OK)
     return st;
-  return launch_gemm<kModeFwd>(X, M, Wq, hl, B, r, Y, sp, d->sms, stream);
+  return launch_gemm<kModeFwd>(X, M, Wq, hl, B, r, Y, sp, d->units, stream);
 }
 
 qlora_status linear_bwd_impl(const uint16_t *dY, const uint16_t *X, const float *XA, int64_t M,
@@ -756,7 +880,7 @@ qlora_status linear_bwd_impl(const uint16_t *dY, const uint16_t *X, const float 
   DeviceInfo *d = nullptr;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t N = Wq->rows, K = Wq->cols;
-  const size_t need = bwd_workspace(M, N, K, r, d->sms) + (keep ? mask_workspace(M, K) : 0);
+  const size_t need = bwd_workspace(M, N, K, r, d->units) + (keep ? mask_workspace(M, K) : 0);
   if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
   Workspace ws{static_cast<char *>(workspace), 0, workspace_bytes};
   const uint16_t *xin = X;
@@ -776,7 +900,7 @@ qlora_status linear_bwd_impl(const uint16_t *dY, const uint16_t *X, const float 
   float *xa_ws = static_cast<float *>(ws.take(static_cast<size_t>(M) * r * 4));
   SplitScratch sp;
   if (!AT || !G || !ghl || !ghlT || !xahlT || !xa_ws) return QLORA_ERR_WORKSPACE;
-  if (dX && !take_split(ws, gemm_split(M, K, N, d->sms), sp)) return QLORA_ERR_WORKSPACE;
+  if (dX && !take_split(ws, gemm_plan(M, K, N, d->units), sp)) return QLORA_ERR_WORKSPACE;
   // s*XA hi|lo transposed [2r, M] (from the saved XA, or recomputed from the adapter input)
   if (XA) {
     if ((st = launch_hilo_t(XA, M, r, s, xahlT, d->sms, stream)) != QLORA_OK) return st;
@@ -790,7 +914,7 @@ qlora_status linear_bwd_impl(const uint16_t *dY, const uint16_t *X, const float 
   // split counters
   if ((st = launch_projection(dY, M, N, B, r, s, G, ghl, ghlT, d->sms, stream, &sp)) != QLORA_OK) return st;
   if (dX) {
-    if ((st = launch_gemm<kModeDx>(dY, M, Wq, ghl, A, r, dX, sp, d->sms, stream, keep, xscale)) != QLORA_OK)
+    if ((st = launch_gemm<kModeDx>(dY, M, Wq, ghl, A, r, dX, sp, d->units, stream, keep, xscale)) != QLORA_OK)
       return st;
   }
   // dA = (1/(1-p)) X_kept^T (s G)  [K, r];  dB = (s XA)^T dY  [r, N]
@@ -907,10 +1031,10 @@ qlora_status qlora_nf4_dequant(const qlora_nf4_t *Wq, uint16_t *W_out, qlora_str
 
 size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
   if (M < 1 || N < 1 || K < 1 || r < 1) return 0;
-  int sms = 148;
+  GemmUnits u;
   DeviceInfo *d = nullptr;
-  if (device_info(&d) == QLORA_OK) sms = d->sms;
-  const size_t f = fwd_workspace(M, N, K, r, sms), b = bwd_workspace(M, N, K, r, sms);
+  if (device_info(&d) == QLORA_OK) u = d->units;
+  const size_t f = fwd_workspace(M, N, K, r, u), b = bwd_workspace(M, N, K, r, u);
   return f > b ? f : b;
 }
 
@@ -1037,6 +1161,17 @@ uint32_t qlora_set_wait_limit_us(uint32_t limit_us) {
   return g_wait_limit_us.exchange(limit_us);
 }
 
+int qlora_set_gemm_pairing(int enable) { return g_gemm_pairing.exchange(enable ? 1 : 0); }
+
+qlora_status qlora_gemm_units(int *ctas, int *pairs) {
+  DeviceInfo *d = nullptr;
+  const qlora_status st = device_info(&d);
+  if (st != QLORA_OK) return st;
+  if (ctas) *ctas = d->units.ctas;
+  if (pairs) *pairs = d->units.pairs;
+  return QLORA_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------ wait self-test
@@ -1106,7 +1241,7 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t *X, int64_t M, c
   if ((st = check_linear_shape(M, Wq, r)) != QLORA_OK) return st;
   DeviceInfo *d = nullptr;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  if (fwd_workspace(M, Wq->rows, Wq->cols, r, d->sms) > kNoallocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (fwd_workspace(M, Wq->rows, Wq->cols, r, d->units) > kNoallocScratchBytes) return QLORA_ERR_WORKSPACE;
   void *scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != QLORA_OK) return st;
   return qlora_linear_fwd(X, M, Wq, A, B, r, s, Y, XA_out, scratch, kNoallocScratchBytes, stream);

@@ -292,6 +292,29 @@ qlora_status qlora_selftest_wait_timeout(uint32_t timeout_us, qlora_stream_t str
 uint32_t qlora_set_wait_limit_us(uint32_t limit_us);
 
 /*
+ * Shape of the fused GEMM launches (forward Y and backward dX).  With pairing on
+ * (the default), a launch whose output width (N forward, K for dX) is a multiple
+ * of 256 runs as clusters of two CTAs that share each 256-row weight tile x
+ * 256-token tile (one M = 256 tensor-core product over both CTAs' shared memory);
+ * other widths, and every launch with pairing off, use one CTA per 128-row tile.
+ * Both shapes accumulate each output over the same K steps in the same order;
+ * only the last-wave split (which tiles of the last round are divided into two
+ * contraction halves, summed in fp32) depends on the shape, so results may differ
+ * by one bf16 ulp between the shapes, and each shape is deterministic.
+ * Process-wide, read once per call; workspace sizes cover either shape.
+ * Returns the previous setting (0 or 1).
+ */
+int qlora_set_gemm_pairing(int enable);
+
+/*
+ * Persistent units of the fused GEMM on the current device: *ctas single CTAs (the
+ * SM count) and *pairs CTA pairs that the device can hold at once (0 when it cannot
+ * place clusters of two).  Either pointer may be NULL.  QLORA_ERR_NO_DEVICE
+ * without a B200-class device.
+ */
+qlora_status qlora_gemm_units(int *ctas, int *pairs);
+
+/*
  * Kernel timing for measurement tools.  While enabled, the library records a
  * pair of CUDA events on the launching stream around every launch of its own
  * kernels, in a ring of QLORA_PROFILE_CAP entries (the oldest entries are
