@@ -49,6 +49,7 @@ WORKLOAD = WORKLOAD_TEXT[HEADLINE]
 FLUSH_BYTES = 256 << 20
 SKINNY = [(m, n, 4096) for n in (4096, 11008) for m in (1, 4, 16)]
 BIG_N = 1_000_000_000
+MERGE_SHAPE = (22016, 8192, 64)  # merge subpath: W [N, K] and adapter rank
 GRAPH_STREAM_BYTES = 320 << 20   # weights streamed per graph replay of the decode measurement
 SMALL_CALLS = 50
 
@@ -750,6 +751,36 @@ def hbm_subpaths(q, torch, dev, stream, P, flush):
     out["dequant_1e9"] = {"ms": td, "GB/s": nbytes / td / 1e6, "frac": nbytes / td / 1e6 / P["hbm"],
                           "bytes": nbytes}
     del W, Wq, out_bf
+    torch.cuda.empty_cache()
+    # merge of a trained adapter into a 16-bit weight (the serving export), from the NF4
+    # base and from the bf16 original: W 22016 x 8192 (the 65B up-projection), r = 64;
+    # L2 flushed before each call
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+    N, K, r = MERGE_SHAPE
+    Wb = (torch.randn(N, K, generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+    Wq = q.nf4_quantize(Wb)
+    A = (torch.randn(K, r, generator=gen, device=dev) / r).to(torch.bfloat16)
+    B = (torch.randn(r, N, generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+    Wm = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    for base in ("nf4", "bf16"):
+        kw = {"Wq": Wq} if base == "nf4" else {"W16": Wb}
+        for _ in range(2):
+            q.nf4_merge(A, B, 0.25, out=Wm, **kw)
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(5):
+            flush.fill_(float(i))
+            q.profile_enable(True)
+            q.nf4_merge(A, B, 0.25, out=Wm, **kw)
+            prof, _ = q.profile_read()
+            q.profile_enable(False)
+            ts += [ms for k, ms in prof if k == "merge"]
+        t = min(ts)
+        by = (Wq.nbytes if base == "nf4" else 2 * N * K) + 2 * N * K + 2 * K * r + 2 * r * N
+        out[f"merge_{base}_{N}x{K}_r{r}"] = {"ms": t, "GB/s": by / t / 1e6, "frac": by / t / 1e6 / P["hbm"],
+                                             "bytes": by}
+    del Wb, Wq, Wm
     torch.cuda.empty_cache()
     # skinny forward: M in {1,4,16}, L2 flushed before each call, whole call timed
     gen = torch.Generator(device=dev)

@@ -20,9 +20,6 @@ using namespace qlora;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
-#ifndef QLORA_GEMM_RASTER_MB
-#define QLORA_GEMM_RASTER_MB 40
-#endif
 constexpr int64_t kSkinnyMaxTokens = 16;   // forward with at most this many tokens: one-launch kernel
 std::atomic<uint32_t> g_wait_limit_us{2000000u};
 std::atomic<int> g_gemm_pairing{1};        // CTA-pair GEMM where the output width allows it
@@ -98,7 +95,7 @@ qlora_status device_info(DeviceInfo **out) {
         set_skinny_attrs<4>() != cudaSuccess || set_skinny_attrs<8>() != cudaSuccess ||
         set_skinny_attrs<16>() != cudaSuccess ||
         cudaFuncSetAttribute(nf4_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             merge_smem_bytes(2)) != cudaSuccess)
+                             merge_smem_max()) != cudaSuccess)
       return QLORA_ERR_CUDA;
     d.units.ctas = d.sms;
     d.units.pairs = 0;
@@ -750,9 +747,14 @@ qlora_status launch_gemm(const uint16_t *act, int64_t M, const qlora_nf4_t *Wq,
   p.num_m_tiles = static_cast<int>((M + kBN - 1) / kBN);
   p.num_w_tiles = static_cast<int>(n_out / (pair ? 2 * kWT : kWT));
   {
-    // token tiles per raster group: as many activation tiles as fit a share of L2
+    // token tiles per raster group.  A packed weight that fits the budget stays in L2
+    // while every token tile sweeps it (one group of one); a larger one is swept by
+    // groups of as many activation tiles as fit the budget, each weight tile read once
+    // per group.
+    constexpr int64_t budget = 40ll << 20;   // bytes of L2 for the group's activation tiles
+    const int64_t w_bytes = n_out * contraction / 2;
     const int64_t act_tile = static_cast<int64_t>(kBN) * contraction * 2;
-    int64_t g = static_cast<int64_t>(QLORA_GEMM_RASTER_MB) * (1 << 20) / act_tile;
+    int64_t g = (w_bytes <= budget) ? 1 : budget / act_tile;
     if (g < 1) g = 1;
     if (g > p.num_m_tiles) g = p.num_m_tiles;
     p.group_m = static_cast<int>(g);
@@ -1093,27 +1095,36 @@ qlora_status qlora_nf4_merge(const qlora_nf4_t *Wq, const uint16_t *W16, int64_t
   if (st != QLORA_OK) return st;
   MergeParams p{};
   if (Wq) {
-    p.codes = Wq->codes;
     p.q8 = Wq->q8;
     p.step = Wq->step;
   }
-  p.w16 = W16;
-  p.out = W_out;
+  p.nf4 = Wq ? 1 : 0;
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.stages = (r + 63) / 64;
   p.s = s;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
   std::memcpy(p.levels, nf4_tables().levels, sizeof(p.levels));
-  CUtensorMap tm_bt, tm_a;
+  CUtensorMap tm_bt, tm_a, tm_base, tm_out;
   // B [r, N]: x = n (inner), y = j; A [K, r]: x = j (inner), y = k.  Boxes reach j = 64 per
-  // stage; rows j >= r are outside the tensors and arrive as zeros.
+  // stage; rows j >= r are outside the tensors and arrive as zeros.  The base: W16
+  // [N, K] in boxes {64 k, 128 n}, or the packed codes [N, K/2 bytes] in boxes
+  // {128 bytes, 128 n}; the output [N, K] in boxes {64 k, 128 n}; all 128B-swizzled.
   if (!make_map_2d(&tm_bt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, r * 2, 64, kMgCols, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, r * 2, 64, kMgCols, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_out, K, N, K * 2, 64, kMgRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
+  const bool base_ok =
+      Wq ? make_map_2d(&tm_base, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, K / 2, N, K / 2, 128, kMgRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B)
+         : make_map_2d(&tm_base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W16, K, N, K * 2, 64, kMgRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!base_ok) return QLORA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((K + kMgCols - 1) / kMgCols), static_cast<unsigned>((N + kMgRows - 1) / kMgRows));
   LaunchTimer lt(QLORA_K_MERGE, stream);
-  nf4_merge_kernel<<<grid, kMgThreads, merge_smem_bytes(p.stages), stream>>>(tm_bt, tm_a, p);
+  nf4_merge_kernel<<<grid, kMgThreads, merge_smem_bytes(p.stages, Wq != nullptr), stream>>>(tm_bt, tm_a, tm_base,
+                                                                                            tm_out, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
 
   uint16_t *sB = reinterpret_cast<uint16_t *>(sm + p.off_b);       // [r][R]
   uint16_t *sX = reinterpret_cast<uint16_t *>(sm + p.off_x);       // [M][xp]
-  float *sRecv = reinterpret_cast<float *>(sm + p.off_part);       // [C ranks][R rows][16 tokens]
+  float *sRecv = reinterpret_cast<float *>(sm + p.off_part);       // [C ranks][R rows][M tokens]
   float *sXA = reinterpret_cast<float *>(sm + p.off_xa);           // [M][r]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + p.off_bar);   // [nmb] codes, then one for B
   uint64_t *bar_b = bars + (p.ks / kSkMacro);
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
     for (int h = 0; h < 2; ++h) {
       const int row = h ? rb : ra;
       const uint32_t owner = static_cast<uint32_t>(row / R);
-      const uint32_t base = recv + 4u * static_cast<uint32_t>((static_cast<int>(rank) * R + row % R) * 16);
+      const uint32_t base = recv + 4u * static_cast<uint32_t>((static_cast<int>(rank) * R + row % R) * p.M);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kSkThreads, 3) qlora_skinny_kernel(
     const int tk = i / R, rr = i - tk * R;
     float v = 0.f;
 #pragma unroll
-    for (int q = 0; q < C; ++q) v += sRecv[(q * R + rr) * 16 + tk];
+    for (int q = 0; q < C; ++q) v += sRecv[(q * R + rr) * p.M + tk];
     float lora = 0.f;
     for (int j = 0; j < p.r; ++j)
       lora = fmaf(sXA[tk * p.r + j], __uint_as_float(static_cast<uint32_t>(sB[j * R + rr]) << 16), lora);
@@ -410,7 +410,7 @@ inline bool skinny_plan_for(int M, int K, int r, int C, int limit, SkinnyPlan &p
   int off = (pl.ks / kSkMacro) * kSkBoxBytes;
   pl.off_b = off;    off += (r * (kSkRows / C) * 2 + 127) & ~127;
   pl.off_x = off;    off += up16(M * pl.xpitch * 2);
-  pl.off_part = off; off += kSkRows * 16 * 4;
+  pl.off_part = off; off += up16(kSkRows * M * 4);   // sized by the tokens: a smaller CTA fits more per SM
   pl.off_xa = off;   off += up16(M * r * 4);
   pl.off_bar = off;  off += 8 * nbars + 16;
   pl.smem = off + 1024;                          // slack for aligning the base to 1024 bytes
