@@ -564,11 +564,16 @@ def main():
                     help="M,N,K[,r]: small profiling case (two fwd+bwd of one projection), no JSON")
     ap.add_argument("--quant-case", type=int, default=None,
                     help="N: profiling case, quantize + dequant of N heavy-tailed values twice, no JSON")
+    ap.add_argument("--merge-case", default=None,
+                    help="N,K,r: profiling case, the adapter merged into W from the NF4 and the bf16 "
+                         "base, twice each, no JSON")
     args = ap.parse_args()
     if args.case:
         return profile_case(*[int(v) for v in args.case.split(",")])
     if args.quant_case:
         return profile_quant_case(args.quant_case)
+    if args.merge_case:
+        return profile_merge_case(*[int(v) for v in args.merge_case.split(",")])
     args.warmup = max(3, args.warmup)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -726,6 +731,28 @@ def profile_quant_case(n):
     torch.cuda.synchronize()
     code, flags = q.device_status()
     print("quant case", n, "status", code, flags)
+    return 0 if code == 0 else 1
+
+
+def profile_merge_case(N, K, r):
+    """The merge of a seeded adapter into a seeded W [N, K], from the NF4 base then from
+    the bf16 base, twice each, through the public API; the case that the merge ncu
+    capture under profiles/ uses (launch order: nf4, nf4, bf16, bf16)."""
+    import torch
+    import bit_nf4_quantized_19_b200 as q
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2)
+    Wb = (torch.randn(N, K, generator=g, device="cuda") * 0.015).to(torch.bfloat16)
+    Wq = q.nf4_quantize(Wb)
+    A = (torch.randn(K, r, generator=g, device="cuda") / r).to(torch.bfloat16)
+    B = (torch.randn(r, N, generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+    out = torch.empty(N, K, dtype=torch.bfloat16, device="cuda")
+    for kw in ({"Wq": Wq}, {"W16": Wb}):
+        for _ in range(2):
+            q.nf4_merge(A, B, 0.25, out=out, **kw)
+    torch.cuda.synchronize()
+    code, flags = q.device_status()
+    print("merge case", N, K, r, "status", code, flags)
     return 0 if code == 0 else 1
 
 
