@@ -24,6 +24,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 QLORA_ERR_TIMEOUT = 5
 DEVSTAT_TIMEOUT = 1
 DEVSTAT_NONFINITE = 2
+DEVSTAT_LAYOUT = 4
 
 
 class QloraError(RuntimeError):

@@ -18,6 +18,7 @@ __device__ uint32_t g_device_status = 0;
 
 constexpr uint32_t kStatTimeout = 1u;
 constexpr uint32_t kStatNonFinite = 2u;
+constexpr uint32_t kStatLayout = 4u;
 
 QDEV uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

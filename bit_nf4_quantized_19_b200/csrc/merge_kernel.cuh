@@ -53,9 +53,11 @@ __host__ __device__ inline int merge_base_bytes(int stages, bool nf4) {
   return kMgCodeBytes + (ops >= 4 * kMgBoxBytes ? 0 : 4 * kMgBoxBytes - ops);
 }
 // At least 80 KB, so at most two CTAs share an SM and their 256 TMEM columns each
-// always fit in the SM's 512.
+// always fit in the SM's 512.  The dynamic shared memory is declared 1024-byte
+// aligned and no slack is reserved for aligning it (the bf16-base plan then fits two
+// CTAs per SM; with slack it missed by 256 bytes); the kernel checks the alignment.
 inline int merge_smem_bytes(int stages, bool nf4) {
-  const int b = 1024 + stages * (kMgABytes + kMgBBytes) + merge_base_bytes(stages, nf4) + 128;
+  const int b = stages * (kMgABytes + kMgBBytes) + merge_base_bytes(stages, nf4) + 128;
   return b < 80 * 1024 ? 80 * 1024 : b;
 }
 inline int merge_smem_max() {
@@ -74,9 +76,14 @@ __global__ void __launch_bounds__(kMgThreads, 1)
     nf4_merge_kernel(const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_out,
                      const __grid_constant__ MergeParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128B-swizzled boxes need 1024-byte alignment, which the declaration asks for
+  // and the plan counts on: a misplaced buffer is reported and nothing is touched
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kStatLayout);
+    return;
+  }
+  uint8_t *smem = smem_raw;
   const int ops_bytes = p.stages * (kMgABytes + kMgBBytes);
   uint8_t *sA = smem;
   uint8_t *sB = sA + p.stages * kMgABytes;

@@ -1136,7 +1136,7 @@ qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags) {
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return QLORA_ERR_CUDA;
   *flags = v;
   if (v & kStatTimeout) return QLORA_ERR_TIMEOUT;
-  if (v & kStatNonFinite) return QLORA_ERR_DEVICE_CHECK;
+  if (v & (kStatNonFinite | kStatLayout)) return QLORA_ERR_DEVICE_CHECK;
   return QLORA_OK;
 }
 

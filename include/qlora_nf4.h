@@ -59,6 +59,7 @@ typedef enum {
 /* Bits of the device status word (qlora_get_device_status). */
 #define QLORA_DEVSTAT_TIMEOUT   1u
 #define QLORA_DEVSTAT_NONFINITE 2u
+#define QLORA_DEVSTAT_LAYOUT    4u   /* a kernel found its shared memory misplaced and did nothing */
 
 /*
  * A quantized weight.  The struct itself lives in host memory; its three arrays
@@ -272,7 +273,8 @@ qlora_status qlora_linear_bwd_ex(const uint16_t *dY, const uint16_t *X, const fl
 /*
  * Synchronizes `stream`, then returns the device status word of the current
  * device in *flags (QLORA_DEVSTAT_* bits) and clears it.  Returns
- * QLORA_ERR_TIMEOUT / QLORA_ERR_DEVICE_CHECK when the corresponding bit was set.
+ * QLORA_ERR_TIMEOUT / QLORA_ERR_DEVICE_CHECK when the corresponding bit was set
+ * (DEVICE_CHECK for NONFINITE and LAYOUT).
  */
 qlora_status qlora_get_device_status(qlora_stream_t stream, uint32_t *flags);
 
