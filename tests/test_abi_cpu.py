@@ -94,6 +94,26 @@ def test_wait_limit_setter_roundtrip(L):
     assert L.qlora_set_wait_limit_us(old) == 123
 
 
+def test_gemm_pairing_setter_roundtrip(L):
+    """The launch-shape switch is process-wide host state: each call returns the
+    previous setting, as 0 or 1."""
+    prev = L.qlora_set_gemm_pairing(0)
+    assert prev in (0, 1)
+    assert L.qlora_set_gemm_pairing(7) == 0
+    assert L.qlora_set_gemm_pairing(prev) == 1
+
+
+def test_gemm_units_without_device(L):
+    """Without a B200 the unit query reports no device and leaves its outputs alone."""
+    import ctypes
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    a, b = ctypes.c_int(-1), ctypes.c_int(-1)
+    assert L.qlora_gemm_units(ctypes.byref(a), ctypes.byref(b)) != 0
+    assert (a.value, b.value) == (-1, -1)
+
+
 def test_plain_c_consumer(L, tmp_path):
     """tests/csrc/abi_consumer.c: a C11 program built with gcc against the header
     alone (-Wall -Wextra -pedantic -Werror) and linked to the shared library runs

@@ -116,3 +116,12 @@ def test_pairing_switch_keeps_workspace_size(q):
     assert q.device_status() == (0, 0)
     assert _apart(H.dev_to_bits(Y1), H.dev_to_bits(Y0), p.K + 2 * p.r) <= 2.0
     assert _apart(H.dev_to_bits(dX1), H.dev_to_bits(dX0), p.N + 2 * p.r) <= 2.0
+
+
+def test_gemm_units_on_device(q):
+    """The single-CTA unit count is the SM count; the pairs the device holds at once
+    are between one and half of it."""
+    import torch
+    ctas, pairs = q.gemm_units()
+    assert ctas == torch.cuda.get_device_properties(0).multi_processor_count
+    assert 1 <= pairs <= ctas // 2
