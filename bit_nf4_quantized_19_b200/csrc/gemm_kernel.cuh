@@ -14,7 +14,7 @@
 // and the weight side repeats B^T (or A) twice, so the adapter term is
 // accumulated to ~2^-16 relative precision, not bf16 precision.
 //
-// Warp roles (512 threads, one CTA per SM, persistent over tiles):
+// Warp roles (640 threads, one CTA per SM, persistent over tiles):
 //   warp 0        TMA producer of the activation tiles (X / dY, or the LoRA
 //                 hi/lo operand).
 //   warp 1        TMEM allocator and single-thread MMA issuer.
@@ -25,7 +25,7 @@
 //                 constants RN32(q8 * step) from the 8-bit codes and the fp32
 //                 group constants (requested one own stage ahead) next to them.
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global (masked rows).
-//   warps 8..15   dequant producers, two warpgroups taking alternate stages:
+//   warps 8..19   dequant producers, three warpgroups taking every third stage:
 //                 packed codes + block constant -> bf16 tile in the
 //                 128-byte-swizzled UMMA layout (one 64-value block per
 //                 thread, decoded through a 16-entry table held in registers),
@@ -61,7 +61,7 @@
 
 namespace qlora {
 
-constexpr int kGemmThreads = 512;
+constexpr int kGemmThreads = 640;
 constexpr int kBN = 256;                  // tokens per tile (MMA N)
 constexpr int kWT = 128;                  // weight-side rows per tile (MMA M)
 constexpr int kBK = 64;                   // contraction per stage (one quant block)
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequant producers
     const int t = (tid - 256) & 127;    // row slot within the stage
-    const int grp = (tid - 256) >> 7;   // warpgroup 0 takes even stages, 1 odd
+    const int grp = (tid - 256) >> 7;   // warpgroup g takes the stages a with a mod 3 = g
     float L[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) L[i] = sL[i];
@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool main = j < nmain;
         const uint32_t my_w = w_cnt;
         if (main) ++w_cnt;
-        if ((a_cnt & 1u) != static_cast<uint32_t>(grp)) continue;
+        if ((a_cnt % 3u) != static_cast<uint32_t>(grp)) continue;
         const int as = static_cast<int>(a_cnt % kStages);
         const uint32_t aph = (a_cnt / kStages) & 1u;
         if (main) {
