@@ -31,9 +31,10 @@ constexpr int kLmABytes = kLmRows * 128;   // 16 KB per stage
 struct LoraMmaParams {
   int rows;              // output rows (tokens for projections, features for gradients)
   int nn;                // MMA N: multiple of 16, <= 256
-  int stages_total;      // contraction stages of 64
-  int stages_per_split;
+  int stages_total;      // contraction steps of 64
+  int stages_per_split;  // steps of 64 per split
   int num_stages;        // smem ring depth
+  int sub;               // steps of 64 per ring slot (one wait, one expect_tx, sub TMA boxes)
   uint32_t tmem_cols;    // power of two >= max(32, nn)
   int splits;            // cluster size along the contraction
   int grad;              // 0: projection outputs, 1: gradient outputs
@@ -71,8 +72,8 @@ constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of
 // shared-memory banks.
 inline __host__ __device__ int lm_partial_pitch(int nn) { return nn + 1; }
 
-inline int lora_mma_smem_bytes(int nn, int stages) {
-  return 1024 + stages * (kLmABytes + nn * 128) + 256;
+inline int lora_mma_smem_bytes(int nn, int stages, int sub) {
+  return 1024 + stages * sub * (kLmABytes + nn * 128) + 256;
 }
 
 QDEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
@@ -92,9 +93,10 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int S = p.num_stages;
   const int b_bytes = p.nn * 128;
+  const int a_slot = p.sub * kLmABytes, b_slot = p.sub * b_bytes;
   uint8_t *sA = smem;
-  uint8_t *sB = sA + S * kLmABytes;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sB + S * b_bytes);
+  uint8_t *sB = sA + S * a_slot;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sB + S * b_slot);
   uint64_t *empty = full + S;
   uint64_t *done = empty + S;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   const int st0 = split * p.stages_per_split;
   const int st1 = min(p.stages_total, st0 + p.stages_per_split);
   const int nst = st1 - st0;
+  const int nslot = (nst + p.sub - 1) / p.sub;   // ring slots this split fills
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -138,17 +141,22 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     uint32_t armed = 0, last = 0;
     int s = 0;
     uint32_t ph = 0;
-    for (int i = 0; i < nst; ++i) {
+    for (int i = 0; i < nslot; ++i) {
       if (!wait_bar(&empty[s], ph ^ 1u, wt)) break;
-      const int c0 = (st0 + i) * 64;
-      mbar_arrive_expect_tx(&full[s], kLmABytes + b_bytes);
-      if (A_MN) {
-        tma_load_2d(sA + s * kLmABytes, map_act, &full[s], row0, c0);
-        tma_load_2d(sA + s * kLmABytes + 8192, map_act, &full[s], row0 + 64, c0);
-      } else {
-        tma_load_2d(sA + s * kLmABytes, map_act, &full[s], c0, row0);
+      const int k0 = st0 + i * p.sub;
+      const int ns = min(p.sub, st1 - k0);
+      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ns * (kLmABytes + b_bytes)));
+      for (int j = 0; j < ns; ++j) {
+        const int c0 = (k0 + j) * 64;
+        uint8_t *da = sA + s * a_slot + j * kLmABytes;
+        if (A_MN) {
+          tma_load_2d(da, map_act, &full[s], row0, c0);
+          tma_load_2d(da + 8192, map_act, &full[s], row0 + 64, c0);
+        } else {
+          tma_load_2d(da, map_act, &full[s], c0, row0);
+        }
+        tma_load_2d(sB + s * b_slot + j * b_bytes, map_q, &full[s], c0, 0);
       }
-      tma_load_2d(sB + s * b_bytes, map_q, &full[s], c0, 0);
       armed |= 1u << s;
       last = (last & ~(1u << s)) | (ph << s);
       if (++s == S) { s = 0; ph ^= 1u; }
@@ -162,16 +170,19 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int i = 0; i < nst; ++i) {
+    for (int i = 0; i < nslot; ++i) {
       if (!wait_bar(&full[s], ph, wt)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t a = smem_u32(sA + s * kLmABytes);
-      const uint32_t b = smem_u32(sB + s * b_bytes);
+      const int ns = min(p.sub, st1 - (st0 + i * p.sub));
+      for (int j = 0; j < ns; ++j) {
+        const uint32_t a = smem_u32(sA + s * a_slot + j * kLmABytes);
+        const uint32_t b = smem_u32(sB + s * b_slot + j * b_bytes);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t ad = A_MN ? sw128_desc(a + k * 2048, 8192, 1024) : sw128_desc(a + k * 32, 16, 1024);
-        const uint64_t bd = sw128_desc(b + k * 32, 16, 1024);
-        mma_bf16_ss(tmem_base, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = A_MN ? sw128_desc(a + k * 2048, 8192, 1024) : sw128_desc(a + k * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(b + k * 32, 16, 1024);
+          mma_bf16_ss(tmem_base, ad, bd, idesc, (i > 0 || j > 0 || k > 0) ? 1u : 0u);
+        }
       }
       mma_commit(&empty[s]);
       if (++s == S) { s = 0; ph ^= 1u; }

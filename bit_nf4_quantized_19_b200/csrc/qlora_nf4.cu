@@ -222,9 +222,19 @@ struct Workspace {
 
 // ---- launch geometry of the rank-r contractions (lora_mma_kernel)
 constexpr int kLmMaxSplits = kLmClusterMax;
+// Ring geometry of the rank-r launches: steps of 64 per ring slot, the ring's byte
+// budget and the fewest slots, for the projections (K-major) and the gradients.
+// Measured on the 65B-shaped step: two steps per slot and a 192 KB ring took the
+// projections from 466 to 417 us per step; the same geometry made the gradients
+// slower (305 to 329 us), so they keep one step per slot in a 110 KB ring.
+struct LmRing {
+  int sub, bytes, min_slots;
+};
+constexpr LmRing kLmRingProject{2, 192 * 1024, 2};
+constexpr LmRing kLmRingGrad{1, 110 * 1024, 3};
 
 struct LmGeom {
-  int nn, row_tiles, stages_total, sps, splits, num_stages;
+  int nn, row_tiles, stages_total, sps, splits, num_stages, sub;
   uint32_t tmem_cols;
 };
 
@@ -272,11 +282,13 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   uint32_t tc = 32;
   while (tc < static_cast<uint32_t>(nn)) tc <<= 1;
   g.tmem_cols = tc;
-  const int stage_bytes = kLmABytes + nn * 128;
+  const LmRing ring = A_MN ? kLmRingGrad : kLmRingProject;
+  g.sub = ring.sub;
+  const int stage_bytes = g.sub * (kLmABytes + nn * 128);
   // the operand ring also holds the fp32 partial tile after the main loop
   int st_min = (kLmRows * lm_partial_pitch(nn) * 4 + stage_bytes - 1) / stage_bytes;
-  if (st_min < 3) st_min = 3;
-  int st_max = (110 * 1024) / stage_bytes;
+  if (st_min < ring.min_slots) st_min = ring.min_slots;
+  int st_max = ring.bytes / stage_bytes;
   if (st_max > 8) st_max = 8;
   if (st_max < st_min) st_max = st_min;
   int64_t best_waves = -1;
@@ -286,7 +298,7 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
     const int sps = (total + c - 1) / c;
     const int splits = (total + sps - 1) / sps;
     for (int S = st_max; S >= st_min; --S) {
-      int active = lm_max_clusters<A_MN>(splits, lora_mma_smem_bytes(nn, S));
+      int active = lm_max_clusters<A_MN>(splits, lora_mma_smem_bytes(nn, S, g.sub));
       if (active <= 0) active = (2 * sms) / splits;   // the runtime could not say
       if (active <= 0) continue;
       const int64_t waves = (g.row_tiles + active - 1) / active;
@@ -454,10 +466,11 @@ qlora_status launch_lora_mma(const LmOperands &o, int64_t contraction, int nn, L
   p.stages_total = g.stages_total;
   p.stages_per_split = g.sps;
   p.num_stages = g.num_stages;
+  p.sub = g.sub;
   p.tmem_cols = g.tmem_cols;
   p.splits = g.splits;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
-  const int smem = lora_mma_smem_bytes(nn, g.num_stages);
+  const int smem = lora_mma_smem_bytes(nn, g.num_stages, g.sub);
   if (smem > 200 * 1024) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(g.row_tiles), static_cast<unsigned>(g.splits), 1);
