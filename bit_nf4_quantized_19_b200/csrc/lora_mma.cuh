@@ -71,6 +71,10 @@ constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of
 // that both a warp over 32 rows of one column and a warp along one row hit 32 distinct
 // shared-memory banks.
 inline __host__ __device__ int lm_partial_pitch(int nn) { return nn + 1; }
+inline __host__ __device__ int lm_partial_bytes(int nn) { return kLmRows * lm_partial_pitch(nn) * 4; }
+// Shared memory the projection epilogue needs after the main loop: the partial tile and
+// the stage of the transposed hi|lo halves (2r <= 2 nn rows of at most 128 + 2 values).
+inline __host__ __device__ int lm_epilogue_bytes(int nn) { return lm_partial_bytes(nn) + 2 * nn * (kLmRows + 2) * 2; }
 
 inline int lora_mma_smem_bytes(int nn, int stages, int sub) {
   return 1024 + stages * sub * (kLmABytes + nn * 128) + 256;
@@ -231,46 +235,81 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const int nr = max(0, r1 - r0);
     const uint32_t base = smem_u32(smem);
     const int pitch = lm_partial_pitch(p.nn);
-    for (int i = tid; i < nr * p.r; i += kLmThreads) {
-      int rr, j;
-      if (p.grad && layout == 0) { rr = i / p.r; j = i - rr * p.r; }     // j fastest: out[row][j]
-      else { j = i / nr; rr = i - j * nr; }                               // row fastest
-      const int rl = r0 + rr, row = row0 + rl;
-      if (row >= rows) continue;
-      const uint32_t a = base + 4u * static_cast<uint32_t>(rl * pitch + j);
-      // every rank's load is issued before the sum, which runs in rank order
-      float pa[kLmClusterMax];
-#pragma unroll
-      for (int qq = 0; qq < kLmClusterMax; ++qq)
-        pa[qq] = qq < p.splits ? ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) : 0.f;
-      float v = 0.f;
-      if (p.grad) {
+    if (p.grad) {
+      for (int i = tid; i < nr * p.r; i += kLmThreads) {
+        int rr, j;
+        if (layout == 0) { rr = i / p.r; j = i - rr * p.r; }     // j fastest: out[row][j]
+        else { j = i / nr; rr = i - j * nr; }                     // row fastest: out[j][row]
+        const int rl = r0 + rr, row = row0 + rl;
+        if (row >= rows) continue;
+        const uint32_t a = base + 4u * static_cast<uint32_t>(rl * pitch + j);
         const uint32_t b = a + 4u * static_cast<uint32_t>(p.r);
-        float pb[kLmClusterMax];
+        // every rank's load is issued before the sum, which runs in rank order
+        float pa[kLmClusterMax], pb[kLmClusterMax];
 #pragma unroll
-        for (int qq = 0; qq < kLmClusterMax; ++qq)
+        for (int qq = 0; qq < kLmClusterMax; ++qq) {
+          pa[qq] = qq < p.splits ? ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) : 0.f;
           pb[qq] = qq < p.splits ? ld_dsmem_f32(map_rank(b, static_cast<uint32_t>(qq))) : 0.f;
+        }
+        float v = 0.f;
 #pragma unroll
         for (int qq = 0; qq < kLmClusterMax; ++qq)
           if (qq < p.splits) v += pa[qq] + pb[qq];
         v = __fmul_rn(v, out_scale);
         float *o = (layout == 0) ? out + static_cast<int64_t>(row) * p.r + j : out + static_cast<int64_t>(j) * rows + row;
         *o = p.accumulate ? __fadd_rn(*o, v) : v;
-      } else {
+      }
+    } else {
+      // Projection: j fastest, so the fp32 result and the row-major hi|lo halves go out
+      // in whole rows; the transposed halves are staged in shared memory ([2r][nr],
+      // after this CTA's own partial tile, which the peers may still be reading) and
+      // written row by row once the rank's rows are done.
+      uint16_t *stT = reinterpret_cast<uint16_t *>(smem + lm_partial_bytes(p.nn));
+      const int tp = nr + 2;   // odd word pitch: a warp's stores along j hit distinct banks
+      const int total = nr * p.r;
+      for (int i0 = tid; i0 < total; i0 += 2 * kLmThreads) {
+        // two elements per pass: all their loads are issued before either sum
+        float pa[2][kLmClusterMax];
 #pragma unroll
-        for (int qq = 0; qq < kLmClusterMax; ++qq)
-          if (qq < p.splits) v += pa[qq];
-        v = __fmul_rn(v, out_scale);
-        if (out) out[static_cast<int64_t>(row) * p.r + j] = v;
-        uint16_t h, l;
-        split_hilo(p.s * v, h, l);
-        if (p.hl) {
-          p.hl[static_cast<int64_t>(row) * 2 * p.r + j] = h;
-          p.hl[static_cast<int64_t>(row) * 2 * p.r + p.r + j] = l;
+        for (int u = 0; u < 2; ++u) {
+          const int i = i0 + u * kLmThreads;
+          const int rr = i / p.r, j = i - rr * p.r;
+          const uint32_t a = base + 4u * static_cast<uint32_t>((r0 + rr) * pitch + j);
+#pragma unroll
+          for (int qq = 0; qq < kLmClusterMax; ++qq)
+            pa[u][qq] = (i < total && qq < p.splits) ? ld_dsmem_f32(map_rank(a, static_cast<uint32_t>(qq))) : 0.f;
         }
-        if (p.hlT) {
-          p.hlT[static_cast<int64_t>(j) * p.ldT + row] = h;
-          p.hlT[static_cast<int64_t>(p.r + j) * p.ldT + row] = l;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = i0 + u * kLmThreads;
+          if (i >= total) continue;
+          const int rr = i / p.r, j = i - rr * p.r;
+          const int row = row0 + r0 + rr;
+          if (row >= rows) continue;
+          float v = 0.f;
+#pragma unroll
+          for (int qq = 0; qq < kLmClusterMax; ++qq)
+            if (qq < p.splits) v += pa[u][qq];
+          v = __fmul_rn(v, out_scale);
+          if (out) out[static_cast<int64_t>(row) * p.r + j] = v;
+          uint16_t h, l;
+          split_hilo(p.s * v, h, l);
+          if (p.hl) {
+            p.hl[static_cast<int64_t>(row) * 2 * p.r + j] = h;
+            p.hl[static_cast<int64_t>(row) * 2 * p.r + p.r + j] = l;
+          }
+          if (p.hlT) {
+            stT[j * tp + rr] = h;
+            stT[(p.r + j) * tp + rr] = l;
+          }
+        }
+      }
+      if (p.hlT) {
+        __syncthreads();
+        for (int i = tid; i < 2 * p.r * nr; i += kLmThreads) {
+          const int jj = i / nr, rr = i - jj * nr;
+          const int row = row0 + r0 + rr;
+          if (row < rows) p.hlT[static_cast<int64_t>(jj) * p.ldT + row] = stT[jj * tp + rr];
         }
       }
     }

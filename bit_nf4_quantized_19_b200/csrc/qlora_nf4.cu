@@ -285,8 +285,10 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   const LmRing ring = A_MN ? kLmRingGrad : kLmRingProject;
   g.sub = ring.sub;
   const int stage_bytes = g.sub * (kLmABytes + nn * 128);
-  // the operand ring also holds the fp32 partial tile after the main loop
-  int st_min = (kLmRows * lm_partial_pitch(nn) * 4 + stage_bytes - 1) / stage_bytes;
+  // after the main loop the operand ring holds the fp32 partial tile (and, for a
+  // projection, the stage of its transposed hi|lo halves)
+  const int epi_bytes = A_MN ? lm_partial_bytes(nn) : lm_epilogue_bytes(nn);
+  int st_min = (epi_bytes + stage_bytes - 1) / stage_bytes;
   if (st_min < ring.min_slots) st_min = ring.min_slots;
   int st_max = ring.bytes / stage_bytes;
   if (st_max > 8) st_max = 8;
