@@ -11,11 +11,14 @@
 // partial tile in shared memory (reusing its operand ring, idle once the last
 // MMA has committed), and rank q then sums rows [q R, (q+1) R) over the cluster
 // in rank order through distributed shared memory (deterministic, no global
-// scratch) and writes the final outputs.  The activation side is the MMA's A operand:
+// scratch) and writes the final outputs in whole rows (a projection's transposed
+// hi|lo halves through a shared-memory stage).  The activation side is the MMA's A operand:
 //   K-major  (projections): Act = X / dY tile [128 tokens x 64 c], TMA box {64, 128}
 //   MN-major (gradients):   Act^T tile [128 features x 64 tokens] from X / dY
 //                           [tokens, features]: two TMA boxes {64 features, 64 tokens}
 // Q is always K-major [nn rows x 64 c], TMA box {64, nn}.
+// A ring slot holds `sub` such 64-wide steps under one barrier (the projections take
+// two, so each activation row is read 256 contiguous bytes at a time).
 // dA and dB contract over the same tokens, so one launch computes both: the row tiles
 // of the second follow those of the first on the grid.
 // Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 4..7 epilogue.
