@@ -558,46 +558,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (role == 2) __threadfence();
       }
       uint16_t *outc = p.out + w0 + row;
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(acc * kBN + cc * 32),
+      for (int cc = 0; cc < kBN / 16; ++cc) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * kBN + cc * 16),
                            v);
         tmem_wait_ld();
         if (two_acc && w.lora) {
           // this tile's contribution: main + keep * (1/(1-p)) * adapter term, per element;
           // the warp's 32 rows are 32 consecutive input features, one mask word per token
-          const int mb = m0 + cc * 32;
+          const int mb = m0 + cc * 16;
           const int64_t kw = (w0 + q * 32) >> 5;
+          uint32_t lv[16];
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(kBN + cc * 16),
+                             lv);
+          tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t lv[16];
-            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                   static_cast<uint32_t>(kBN + cc * 32 + h * 16),
-                               lv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int m = mb + h * 16 + j;
-              const uint32_t word = (m < p.M) ? __ldg(p.keep32 + static_cast<int64_t>(m) * keep_words + kw) : 0u;
-              if ((word >> lane) & 1u)
-                v[h * 16 + j] = __float_as_uint(__fadd_rn(__uint_as_float(v[h * 16 + j]),
-                                                          __fmul_rn(p.keep_scale, __uint_as_float(lv[j]))));
-            }
+          for (int j = 0; j < 16; ++j) {
+            const int m = mb + j;
+            const uint32_t word = (m < p.M) ? __ldg(p.keep32 + static_cast<int64_t>(m) * keep_words + kw) : 0u;
+            if ((word >> lane) & 1u)
+              v[j] = __float_as_uint(__fadd_rn(__uint_as_float(v[j]), __fmul_rn(p.keep_scale, __uint_as_float(lv[j]))));
           }
         }
         if (role == 1) {
-          float4 *d4 = reinterpret_cast<float4 *>(prow + cc * 32);
+          float4 *d4 = reinterpret_cast<float4 *>(prow + cc * 16);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < 4; ++j)
             d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           continue;
         }
         if (role == 2) {
-          const float4 *s4 = reinterpret_cast<const float4 *>(prow + cc * 32);
+          const float4 *s4 = reinterpret_cast<const float4 *>(prow + cc * 16);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             const float4 f = __ldcg(s4 + j);
             v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + f.x);
             v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + f.y);
@@ -605,9 +601,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + f.w);
           }
         }
-        const int mb = m0 + cc * 32;
+        const int mb = m0 + cc * 16;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const int m = mb + j;
           if (m < p.M) {
             const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[j]));
