@@ -145,3 +145,38 @@ def test_smi_device_id_follows_cuda_visible_devices():
     assert bench.smi_device_id(2, "3,5") == "2"          # out of range: the index itself
     assert bench.smi_device_id(0, "all") == "0"          # not an index or a UUID
     assert bench.smi_device_id(0, "") == "0"
+
+
+def _fake_tree(tmp_path, kernel_text):
+    csrc = tmp_path / "bit_nf4_quantized_19_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "gemm_kernel.cuh").write_text(kernel_text)
+    (csrc / "common.cuh").write_text("// shared helpers\n")
+    (csrc / "qlora_nf4.cu").write_text("qlora_status launch_gemm(int x) {\n  return x;\n}\n")
+    (tmp_path / "profiles").mkdir()
+    return tmp_path
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_captured_on(tmp_path, monkeypatch):
+    root = _fake_tree(tmp_path, "// kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h1 = bench.source_hash("qlora_gemm_kernel")
+    (root / "profiles" / "traffic.json").write_text(
+        json.dumps({"qlora_gemm_kernel": {"source_hash": h1, "bytes_per_launch": 1.5e9}}))
+    assert bench.traffic_for("qlora_gemm_kernel") == 1.5e9
+    # any change to the kernel's header (or its launcher) makes the stored figure stale
+    (root / "bit_nf4_quantized_19_b200" / "csrc" / "gemm_kernel.cuh").write_text("// kernel v2\n")
+    assert bench.source_hash("qlora_gemm_kernel") != h1
+    assert bench.traffic_for("qlora_gemm_kernel") is None
+    (root / "bit_nf4_quantized_19_b200" / "csrc" / "gemm_kernel.cuh").write_text("// kernel v1\n")
+    (root / "bit_nf4_quantized_19_b200" / "csrc" / "qlora_nf4.cu").write_text(
+        "qlora_status launch_gemm(int x) {\n  return x + 1;\n}\n")
+    assert bench.traffic_for("qlora_gemm_kernel") is None
+
+
+def test_traffic_missing_file_or_kernel_reads_null(tmp_path, monkeypatch):
+    root = _fake_tree(tmp_path, "// kernel\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.traffic_for("qlora_gemm_kernel") is None
+    (root / "profiles" / "traffic.json").write_text("{}")
+    assert bench.traffic_for("qlora_gemm_kernel") is None
