@@ -73,13 +73,15 @@ constexpr int kLmClusterMax = 8;   // portable cluster size: at most 8 splits of
 // Row pitch (floats) of the fp32 partial tile staged for the cluster reduction: odd, so
 // that both a warp over 32 rows of one column and a warp along one row hit 32 distinct
 // shared-memory banks.
-inline __host__ __device__ int lm_partial_pitch(int nn) { return nn + 1; }
-inline __host__ __device__ int lm_partial_bytes(int nn) { return kLmRows * lm_partial_pitch(nn) * 4; }
+constexpr __host__ __device__ int lm_partial_pitch(int nn) { return nn + 1; }
+constexpr __host__ __device__ int lm_partial_bytes(int nn) { return kLmRows * lm_partial_pitch(nn) * 4; }
 // Shared memory the projection epilogue needs after the main loop: the partial tile and
 // the stage of the transposed hi|lo halves (2r <= 2 nn rows of at most 128 + 2 values).
-inline __host__ __device__ int lm_epilogue_bytes(int nn) { return lm_partial_bytes(nn) + 2 * nn * (kLmRows + 2) * 2; }
+constexpr __host__ __device__ int lm_epilogue_bytes(int nn) { return lm_partial_bytes(nn) + 2 * nn * (kLmRows + 2) * 2; }
 
-inline int lora_mma_smem_bytes(int nn, int stages, int sub) {
+constexpr int kLmSmemMax = 200 * 1024;   // the kernels' dynamic shared-memory attribute
+
+constexpr int lora_mma_smem_bytes(int nn, int stages, int sub) {
   return 1024 + stages * sub * (kLmABytes + nn * 128) + 256;
 }
 

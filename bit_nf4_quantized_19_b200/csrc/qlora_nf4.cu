@@ -82,9 +82,9 @@ qlora_status device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(qlora_gemm_kernel<kModeDx, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGemmSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if (cudaFuncSetAttribute(lora_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+    if (cudaFuncSetAttribute(lora_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmemMax) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(lora_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+        cudaFuncSetAttribute(lora_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmemMax) !=
             cudaSuccess ||
         cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes) !=
             cudaSuccess ||
@@ -233,6 +233,34 @@ struct LmRing {
 constexpr LmRing kLmRingProject{2, 192 * 1024, 2};
 constexpr LmRing kLmRingGrad{1, 110 * 1024, 3};
 
+// Ring depths a plan may take: at least the ring's fewest slots and enough slots to
+// hold what the epilogue keeps in the idle ring (the fp32 partial tile and, for a
+// projection, the stage of its transposed hi|lo halves); at most the ring's byte
+// budget (and 8 slots), unless the epilogue needs more.
+struct LmSlots {
+  int min, max;
+};
+constexpr LmSlots lm_slots(const LmRing &ring, int nn, bool projection) {
+  const int stage_bytes = ring.sub * (kLmABytes + nn * 128);
+  const int epi_bytes = projection ? lm_epilogue_bytes(nn) : lm_partial_bytes(nn);
+  int lo = (epi_bytes + stage_bytes - 1) / stage_bytes;
+  if (lo < ring.min_slots) lo = ring.min_slots;
+  int hi = ring.bytes / stage_bytes;
+  if (hi > 8) hi = 8;
+  if (hi < lo) hi = lo;
+  return LmSlots{lo, hi};
+}
+// Every plan the host can pick fits the attribute: projections have nn = r rounded up
+// to 16 (r <= 128), gradients nn = 2r.
+constexpr bool lm_plans_fit() {
+  for (int nn = 16; nn <= 128; nn += 16)
+    if (lora_mma_smem_bytes(nn, lm_slots(kLmRingProject, nn, true).max, kLmRingProject.sub) > kLmSmemMax) return false;
+  for (int nn = 16; nn <= 256; nn += 16)
+    if (lora_mma_smem_bytes(nn, lm_slots(kLmRingGrad, nn, false).max, kLmRingGrad.sub) > kLmSmemMax) return false;
+  return true;
+}
+static_assert(lm_plans_fit(), "a rank-r ring plan exceeds the shared-memory attribute");
+
 struct LmGeom {
   int nn, row_tiles, stages_total, sps, splits, num_stages, sub;
   uint32_t tmem_cols;
@@ -284,15 +312,8 @@ LmGeom lm_geom(int64_t rows, int64_t contraction, int nn, int sms) {
   g.tmem_cols = tc;
   const LmRing ring = A_MN ? kLmRingGrad : kLmRingProject;
   g.sub = ring.sub;
-  const int stage_bytes = g.sub * (kLmABytes + nn * 128);
-  // after the main loop the operand ring holds the fp32 partial tile (and, for a
-  // projection, the stage of its transposed hi|lo halves)
-  const int epi_bytes = A_MN ? lm_partial_bytes(nn) : lm_epilogue_bytes(nn);
-  int st_min = (epi_bytes + stage_bytes - 1) / stage_bytes;
-  if (st_min < ring.min_slots) st_min = ring.min_slots;
-  int st_max = ring.bytes / stage_bytes;
-  if (st_max > 8) st_max = 8;
-  if (st_max < st_min) st_max = st_min;
+  const LmSlots slots = lm_slots(ring, nn, !A_MN);
+  const int st_min = slots.min, st_max = slots.max;
   int64_t best_waves = -1;
   for (int c = kLmMaxSplits; c >= 1; c >>= 1) {   // the splits of a tile form one cluster
     if (c > 1 && c > g.stages_total) continue;
@@ -473,7 +494,7 @@ qlora_status launch_lora_mma(const LmOperands &o, int64_t contraction, int nn, L
   p.splits = g.splits;
   p.limit_ns = static_cast<uint64_t>(g_wait_limit_us.load()) * 1000ull;
   const int smem = lora_mma_smem_bytes(nn, g.num_stages, g.sub);
-  if (smem > 200 * 1024) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (smem > kLmSmemMax) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(g.row_tiles), static_cast<unsigned>(g.splits), 1);
   cfg.blockDim = dim3(kLmThreads, 1, 1);
