@@ -97,6 +97,16 @@ static_assert(kGemmSmemBytes <= 227 * 1024, "GEMM shared memory exceeds the per-
 static_assert(GemmShape<true>::kStagesAB <= kMaxStagesAB && GemmShape<false>::kStagesAB <= kMaxStagesAB, "");
 static_assert(kStagesW <= 32 && kMaxStagesAB <= 32, "ring bookkeeping uses 32-bit masks");
 static_assert(kStagesW % 2 == 0, "the two weight producer warps each keep to the slots of one parity");
+static_assert(kGemmThreads == 256 + 3 * 128,
+              "warps 0..7, then three dequant warpgroups; the dequant loop gives stage a to warpgroup a mod 3");
+// A dequant warpgroup's previous stage was a - 3, whose wait needed A stage a - 3 - S
+// consumed; with S >= 3 that covers a - 2S, so its wait on A slot a never sees the
+// barrier two phases behind.  Its wait on W slot w comes after the A slot is free,
+// which needs the W stage kStagesW earlier to map to an A stage at least S back.
+static_assert(GemmShape<false>::kStagesAB >= 3 && GemmShape<true>::kStagesAB >= 3,
+              "the A-slot phase argument needs at least three A stages");
+static_assert(kStagesW >= GemmShape<false>::kStagesAB && kStagesW >= GemmShape<true>::kStagesAB,
+              "the W-slot phase argument needs at least as many W stages as A stages");
 
 enum GemmMode : int { kModeFwd = 0, kModeDx = 1 };
 
