@@ -87,6 +87,22 @@ def test_reference_arm_prints_the_contract_line():
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
 
+@pytest.mark.parametrize("rank", [0, 1])
+def test_reference_arm_under_two_ranks(rank):
+    """Launched as two ranks, the reference arm runs and prints on rank 0 only (n_gpus
+    the world size); the other rank exits 0 without work or output."""
+    env = dict(os.environ, WORLD_SIZE="2", RANK=str(rank), LOCAL_RANK=str(rank))
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3", "--gpus", "2"], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    if rank == 0:
+        line = json.loads(res.stdout.strip().splitlines()[-1])
+        assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    else:
+        assert res.stdout.strip() == ""
+
+
 FAKE_SMI = r'''#!{python}
 import datetime, sys, time
 args = sys.argv[1:]
